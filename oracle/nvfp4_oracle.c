@@ -1,0 +1,444 @@
+/*
+ * nvfp4_oracle.c -- plain, slow CPU oracle for the NVFP4 quantized linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may include, link or
+ * call this file: only tests/, __graft_entry__.smoke() and bench.py's CPU
+ * baseline leg use it.  It shares no code, header, table or constant generator
+ * with the CUDA library; both sides only consume the same seeded input bytes.
+ *
+ * Source of the method: "Pretraining Large Language Models with NVFP4"
+ * (gist.science summary of arXiv 2509.25149), section "Technische samenvatting":
+ *   2A  "Het NVFP4 Formaat"      -- 16-element blocks, E4M3 block scales, an FP32
+ *                                  per-tensor scale on top (two-level scaling);
+ *   2B.2 "Random Hadamard Transforms" -- 16x16 RHT on the inputs of the Wgrad GEMM;
+ *   2B.3 "Twee-dimensionale (2D) Blokschaling" -- 16x16 blocks for weights,
+ *                                  1x16 for activations and gradients;
+ *   2B.4 "Stochastisch Afronden" -- stochastic rounding on gradients only, in
+ *                                  contrast with round-to-nearest-even;
+ * and the lay section "De kern", item "De Gok" (3.4 -> 3 with 60 %, 4 with 40 %).
+ * "NVIDIA acelera el preentrenamiento de LLM: NVFP4 en Blackwell junto con JAX y
+ * MaxText", section "Como Funciona Mixed-Precision con NVFP4": GEMMs take NVFP4
+ * weights and activations, accumulators stay in high precision.
+ *
+ * The pages print no formula beyond the above.  Every precise step below that
+ * they leave open is a reading, tagged R1..R20 as in the design notes:
+ *   R1  E2M1 round-to-nearest, ties to the even code, saturate at 6
+ *   R2  a value that rounds to magnitude 0 encodes as 0x0 (never 0x8)
+ *   R3  E4M3 encode: round-to-nearest-even, saturate to 448 (satfinite)
+ *   R4  S_enc = 2688/A and s_g = A/2688, one IEEE FP32 division each
+ *   R5  A == 0  ->  S_enc = s_g = 1 (all codes and scales come out 0)
+ *   R6  d = (bamax * S_enc) / 6 in FP32, in this order
+ *   R7  the block scale is d rounded to nearest E4M3 (not rounded up)
+ *   R8  a block whose decoded scale is 0 gets all-zero codes
+ *   R9  y = x * (S_enc / s_b), FP32, in this order
+ *   R10 SR: round up iff (w >> 8) * 2^-24 < p, p the fractional position
+ *   R11 Philox4x32-10, key = seed, counter = (idx>>2 lo, idx>>2 hi, domain, 0),
+ *       word idx & 3
+ *   R12 idx = r*C + c, the element's row-major index in the input [R, C]
+ *   R13 domain 0 = row-wise SR, 1 = column-wise SR, 2 = RHT signs
+ *   R14 RHT signs: bit j of word 0 of Philox(key 0, counter (0,0,2,0)); set -> -1
+ *   R15 the RHT acts on aligned 16-runs along the GEMM K dimension (tokens)
+ *   R16 RHT FP32 order: signs, butterflies h = 1,2,4,8, then * 0.25
+ *   R17 packing: element 2i in the low nibble, 2i+1 in the high nibble
+ *   R18 scale layout: 128x4 tiles of 512 bytes (see orc_sf_offset)
+ * Floating point: built with -ffp-contract=off and without fast-math, so every
+ * FP32 operation below is one IEEE operation in the order written.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------ */
+/* Element and scale formats (section 2A: FP4 elements, E4M3 block scales).  */
+/* Decoding follows the bit-field definition of each format; encoding is the */
+/* plain "nearest representable value" search over the decoded values.      */
+/* ------------------------------------------------------------------------ */
+
+/* E2M1: 1 sign, 2 exponent (bias 1), 1 mantissa bit; exponent 0 is subnormal. */
+double orc_e2m1_decode(int code)
+{
+    int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -mag : mag;
+}
+
+/* E4M3: 1 sign, 4 exponent (bias 7), 3 mantissa bits; exponent 0 is subnormal;
+ * S.1111.111 is NaN and there is no infinity. */
+double orc_e4m3_decode(int byte)
+{
+    int s = (byte >> 7) & 1, e = (byte >> 3) & 15, m = byte & 7;
+    if (e == 15 && m == 7) return NAN;
+    double mag = (e == 0) ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* R1, R2: magnitudes at or above 6 saturate to 6; below, the nearest of the
+ * eight magnitudes, and on a tie the even code wins. */
+int orc_e2m1_encode_rn(float y)
+{
+    double a = fabs((double)y);
+    if (a >= 6.0) return (y < 0.0f) ? 0xF : 0x7;
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c < 8; c++) {
+        double dist = fabs(a - orc_e2m1_decode(c));
+        if (dist < bd || (dist == bd && (c & 1) == 0)) { bd = dist; best = c; }
+    }
+    if (best != 0 && y < 0.0f) best |= 8;
+    return best;
+}
+
+/* R3: non-negative d -> nearest finite E4M3 code in [0, 0x7E], ties to the even
+ * code, anything above 448 saturates to 448.  Binary search over the monotone
+ * positive codes, then a nearest-of-two decision. */
+int orc_e4m3_encode_rn_sat(float d)
+{
+    double a = (double)d;
+    if (!(a > 0.0)) return 0;              /* 0, -0 (and NaN: out of contract) */
+    if (a >= 448.0) return 0x7E;
+    int lo = 0, hi = 0x7E;                 /* value(lo) <= a < value(hi) */
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (orc_e4m3_decode(mid) <= a) lo = mid; else hi = mid;
+    }
+    double dl = a - orc_e4m3_decode(lo), dh = orc_e4m3_decode(hi) - a;
+    if (dl < dh) return lo;
+    if (dh < dl) return hi;
+    return (lo & 1) ? hi : lo;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As    */
+/* Easy as 1, 2, 3", SC'11): ten rounds of two 32x32->64 multiplies with the  */
+/* published multipliers, Weyl key schedule between rounds.                  */
+/* ------------------------------------------------------------------------ */
+void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; round++) {
+        if (round > 0) { k0 += 0x9E3779B9u; k1 += 0xBB67AE85u; }
+        uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+        c0 = n0; c1 = lo1; c2 = n2; c3 = lo0;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* R11-R13: the 32-bit word that element idx draws in a given domain. */
+uint32_t orc_sr_word(uint64_t seed, uint64_t idx, uint32_t domain)
+{
+    uint64_t g = idx >> 2;
+    uint32_t ctr[4] = {(uint32_t)g, (uint32_t)(g >> 32), domain, 0u};
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t out[4];
+    orc_philox4x32_10(ctr, key, out);
+    return out[idx & 3];
+}
+
+/* ------------------------------------------------------------------------ */
+/* Rounding of one scaled value y (section 2B.4 and "De Gok").               */
+/* ------------------------------------------------------------------------ */
+
+static int code_of_magnitude(float mag, float y)
+{
+    for (int c = 0; c < 8; c++)
+        if ((double)mag == orc_e2m1_decode(c)) return (c != 0 && y < 0.0f) ? (c | 8) : c;
+    return -1; /* unreachable for magnitudes on the grid */
+}
+
+/* R10: stochastic rounding between the two neighbouring grid magnitudes.
+ * Between 0 and 2 the grid step is 0.5, between 2 and 4 it is 1, between 4 and
+ * 6 it is 2; lo and p are exact in FP32 because each step is a power of two. */
+int orc_e2m1_encode_sr(float y, uint32_t w)
+{
+    float a = fabsf(y);
+    if (a > 6.0f) a = 6.0f;
+    float step = (a < 2.0f) ? 0.5f : ((a < 4.0f) ? 1.0f : 2.0f);
+    float lo = floorf(a / step) * step;
+    float p = (a - lo) / step;
+    float u = (float)(w >> 8) * 0x1p-24f;
+    float mag = (u < p) ? lo + step : lo;
+    return code_of_magnitude(mag, y);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Random Hadamard transform (section 2B.2): Q = 1/4 * H16 * diag(s).        */
+/* ------------------------------------------------------------------------ */
+
+/* R14 */
+void orc_rht_signs(float s[16])
+{
+    uint32_t ctr[4] = {0u, 0u, 2u, 0u}, key[2] = {0u, 0u}, out[4];
+    orc_philox4x32_10(ctr, key, out);
+    for (int j = 0; j < 16; j++) s[j] = ((out[0] >> j) & 1u) ? -1.0f : 1.0f;
+}
+
+/* R16: FP32, fixed order. */
+void orc_rht16_f32(const float x[16], float y[16])
+{
+    float s[16], v[16];
+    orc_rht_signs(s);
+    for (int j = 0; j < 16; j++) v[j] = (s[j] < 0.0f) ? -x[j] : x[j];
+    for (int h = 1; h < 16; h <<= 1)
+        for (int j = 0; j < 16; j++)
+            if ((j & h) == 0) {
+                float a = v[j], b = v[j + h];
+                v[j] = a + b;
+                v[j + h] = a - b;
+            }
+    for (int j = 0; j < 16; j++) y[j] = v[j] * 0.25f;
+}
+
+/* The same transform in FP64 (used only to pin orthogonality). */
+void orc_rht16_f64(const double x[16], double y[16])
+{
+    float s[16];
+    double v[16];
+    orc_rht_signs(s);
+    for (int j = 0; j < 16; j++) v[j] = (s[j] < 0.0f) ? -x[j] : x[j];
+    for (int h = 1; h < 16; h <<= 1)
+        for (int j = 0; j < 16; j++)
+            if ((j & h) == 0) {
+                double a = v[j], b = v[j + h];
+                v[j] = a + b;
+                v[j + h] = a - b;
+            }
+    for (int j = 0; j < 16; j++) y[j] = v[j] * 0.25;
+}
+
+/* ------------------------------------------------------------------------ */
+/* BF16 input and the per-tensor scale (section 2A, first level).           */
+/* ------------------------------------------------------------------------ */
+
+static inline float bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* max |x| over a row-major BF16 [R, C] tensor with row pitch ld (elements). */
+float orc_amax(const uint16_t *x, int64_t R, int64_t C, int64_t ld)
+{
+    float m = 0.0f;
+#pragma omp parallel for reduction(max : m) schedule(static)
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t c = 0; c < C; c++) {
+            float a = fabsf(bf16_to_f32(x[r * ld + c]));
+            if (a > m) m = a;
+        }
+    return m;
+}
+
+/* max |Q x| where Q acts on each aligned 16-run of rows of every column (R15). */
+float orc_amax_rht(const uint16_t *x, int64_t R, int64_t C, int64_t ld)
+{
+    float m = 0.0f;
+#pragma omp parallel for reduction(max : m) schedule(static)
+    for (int64_t tb = 0; tb < R / 16; tb++)
+        for (int64_t c = 0; c < C; c++) {
+            float v[16], y[16];
+            for (int i = 0; i < 16; i++) v[i] = bf16_to_f32(x[(tb * 16 + i) * ld + c]);
+            orc_rht16_f32(v, y);
+            for (int i = 0; i < 16; i++) {
+                float a = fabsf(y[i]);
+                if (a > m) m = a;
+            }
+        }
+    return m;
+}
+
+/* R4, R5.  out[0] = S_enc (encode), out[1] = s_g (decode, exported). */
+void orc_global_scales(float amax, float out[2])
+{
+    if (amax == 0.0f) { out[0] = 1.0f; out[1] = 1.0f; return; }
+    out[0] = 2688.0f / amax;
+    out[1] = amax / 2688.0f;
+}
+
+/* ------------------------------------------------------------------------ */
+/* One block (section 2A, second level): n = 16 (1D) or 256 (2D) values.    */
+/* ------------------------------------------------------------------------ */
+static int quant_block(const float *v, int n, float s_enc, int sr, const uint32_t *words,
+                       uint8_t *codes)
+{
+    float bamax = 0.0f;
+    for (int i = 0; i < n; i++) {
+        float a = fabsf(v[i]);
+        if (a > bamax) bamax = a;
+    }
+    float d = (bamax * s_enc) / 6.0f;                  /* R6 */
+    int sf = orc_e4m3_encode_rn_sat(d);                /* R7 */
+    float sb = (float)orc_e4m3_decode(sf);
+    if (sb == 0.0f) {                                  /* R8 */
+        for (int i = 0; i < n; i++) codes[i] = 0;
+        return sf;
+    }
+    float r = s_enc / sb;                              /* R9 */
+    for (int i = 0; i < n; i++) {
+        float y = v[i] * r;
+        codes[i] = (uint8_t)(sr ? orc_e2m1_encode_sr(y, words[i]) : orc_e2m1_encode_rn(y));
+    }
+    return sf;
+}
+
+/* Row-wise 1x16 quantization (section 2B.3: activations and gradients).
+ * codes: [R, C] one code per byte; sf: [R, C/16]. */
+void orc_quantize_row(const uint16_t *x, int64_t R, int64_t C, int64_t ld, float amax, int sr,
+                      uint64_t seed, uint8_t *codes, uint8_t *sf)
+{
+    float g[2];
+    orc_global_scales(amax, g);
+    int64_t S = C / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t b = 0; b < S; b++) {
+            float v[16];
+            uint32_t w[16];
+            for (int i = 0; i < 16; i++) {
+                int64_t c = b * 16 + i;
+                v[i] = bf16_to_f32(x[r * ld + c]);
+                w[i] = sr ? orc_sr_word(seed, (uint64_t)(r * C + c), 0u) : 0u;
+            }
+            sf[r * S + b] = (uint8_t)quant_block(v, 16, g[0], sr, w, codes + r * C + b * 16);
+        }
+}
+
+/* Column-wise 1x16 quantization along R (the GEMM K dimension of wgrad), with
+ * an optional RHT on each 16-run and optional SR.  The output is the transposed
+ * copy: codes_t [C, R], sf_t [C, R/16].  amax must be the amax of the tensor the
+ * blocks are taken from (orc_amax_rht when rht is set). */
+void orc_quantize_col(const uint16_t *x, int64_t R, int64_t C, int64_t ld, float amax, int rht,
+                      int sr, uint64_t seed, uint8_t *codes_t, uint8_t *sf_t)
+{
+    float g[2];
+    orc_global_scales(amax, g);
+    int64_t S = R / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < C; c++)
+        for (int64_t tb = 0; tb < S; tb++) {
+            float v[16], y[16];
+            uint32_t w[16];
+            uint8_t q[16];
+            for (int i = 0; i < 16; i++) {
+                int64_t r = tb * 16 + i;
+                v[i] = bf16_to_f32(x[r * ld + c]);
+                w[i] = sr ? orc_sr_word(seed, (uint64_t)(r * C + c), 1u) : 0u;
+            }
+            if (rht) orc_rht16_f32(v, y); else memcpy(y, v, sizeof y);
+            sf_t[c * S + tb] = (uint8_t)quant_block(y, 16, g[0], sr, w, q);
+            for (int i = 0; i < 16; i++) codes_t[c * R + tb * 16 + i] = q[i];
+        }
+}
+
+/* 2D 16x16 quantization of a weight W [N, K] (section 2B.3), round to nearest.
+ * codes: [N, K]; sf_tile: [N/16, K/16], one scale per 16x16 tile. */
+void orc_quantize_2d(const uint16_t *w, int64_t N, int64_t K, int64_t ld, float amax,
+                     uint8_t *codes, uint8_t *sf_tile)
+{
+    float g[2];
+    orc_global_scales(amax, g);
+    int64_t TN = N / 16, TK = K / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t bn = 0; bn < TN; bn++)
+        for (int64_t bk = 0; bk < TK; bk++) {
+            float v[256];
+            uint8_t q[256];
+            for (int i = 0; i < 16; i++)
+                for (int j = 0; j < 16; j++)
+                    v[i * 16 + j] = bf16_to_f32(w[(bn * 16 + i) * ld + bk * 16 + j]);
+            sf_tile[bn * TK + bk] = (uint8_t)quant_block(v, 256, g[0], 0, NULL, q);
+            for (int i = 0; i < 16; i++)
+                for (int j = 0; j < 16; j++)
+                    codes[(bn * 16 + i) * K + bk * 16 + j] = q[i * 16 + j];
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Storage layouts (R17, R18).                                              */
+/* ------------------------------------------------------------------------ */
+
+/* R17: codes [R, C] -> bytes [R, C/2]. */
+void orc_pack_nibbles(const uint8_t *codes, int64_t R, int64_t C, uint8_t *packed)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t i = 0; i < C / 2; i++)
+            packed[r * (C / 2) + i] =
+                (uint8_t)((codes[r * C + 2 * i] & 15) | ((codes[r * C + 2 * i + 1] & 15) << 4));
+}
+
+/* R18: byte offset of scale (r, c) in a matrix of Rp = pad128(R) rows and
+ * Sp = pad4(S) scale columns, stored as 128x4 tiles of 512 bytes; inside a tile,
+ * row r sits at (r % 32) * 16 + ((r % 128) / 32) * 4 and column c at c % 4. */
+int64_t orc_sf_offset(int64_t r, int64_t c, int64_t Sp)
+{
+    return ((r / 128) * (Sp / 4) + c / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4);
+}
+
+/* sf [R, S] -> swizzled buffer of pad128(R) * pad4(S) bytes, padding zero. */
+void orc_swizzle_scales(const uint8_t *sf, int64_t R, int64_t S, uint8_t *out)
+{
+    int64_t Rp = (R + 127) / 128 * 128, Sp = (S + 3) / 4 * 4;
+    memset(out, 0, (size_t)(Rp * Sp));
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t c = 0; c < S; c++) out[orc_sf_offset(r, c, Sp)] = sf[r * S + c];
+}
+
+/* ------------------------------------------------------------------------ */
+/* Block-scaled GEMM (FP64 definition):                                      */
+/*   D[m,n] = sum_k dq(A[m,k]) * dq(B[n,k]),  dq = e2m1(code) * e4m3(sf) * s_g */
+/* Unpacked operands: codes [rows, K], scales [rows, K/16].  absum receives   */
+/* sum_k |dq(a) dq(b)| for the error bound.  Either D and absum are full      */
+/* [M, N] (pairs == NULL) or they hold npairs sampled entries (m, n).        */
+/* ------------------------------------------------------------------------ */
+void orc_gemm(const uint8_t *ca, const uint8_t *sa, float sga, const uint8_t *cb,
+              const uint8_t *sb, float sgb, int64_t M, int64_t N, int64_t K,
+              const int64_t *pairs, int64_t npairs, double *D, double *absum)
+{
+    int64_t S = K / 16;
+    int64_t total = pairs ? npairs : M * N;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t t = 0; t < total; t++) {
+        int64_t m = pairs ? pairs[2 * t] : t / N;
+        int64_t n = pairs ? pairs[2 * t + 1] : t % N;
+        double acc = 0.0, aacc = 0.0;
+        for (int64_t k = 0; k < K; k++) {
+            double a = orc_e2m1_decode(ca[m * K + k]) * orc_e4m3_decode(sa[m * S + k / 16]) * (double)sga;
+            double b = orc_e2m1_decode(cb[n * K + k]) * orc_e4m3_decode(sb[n * S + k / 16]) * (double)sgb;
+            acc += a * b;
+            aacc += fabs(a * b);
+        }
+        D[t] = acc;
+        absum[t] = aacc;
+    }
+}
+
+/* dq of a whole unpacked operand: out [R, C] doubles. */
+void orc_dequantize(const uint8_t *codes, const uint8_t *sf, float sg, int64_t R, int64_t C,
+                    double *out)
+{
+    int64_t S = C / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t c = 0; c < C; c++)
+            out[r * C + c] = orc_e2m1_decode(codes[r * C + c]) * orc_e4m3_decode(sf[r * S + c / 16]) * (double)sg;
+}
+
+int orc_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
