@@ -1,0 +1,185 @@
+/*
+ * nvfp4.h -- C ABI of the B200 (sm_100a) NVFP4 quantized linear layer.
+ *
+ * The method: "Pretraining Large Language Models with NVFP4" (gist.science
+ * summary of arXiv 2509.25149), section "Technische samenvatting":
+ *   2A   NVFP4: FP4 (E2M1) values in blocks of 16 with one E4M3 scale per block
+ *        and one FP32 scale per tensor (two-level scaling);
+ *   2B.2 a 16x16 random Hadamard transform on the inputs of the Wgrad GEMM;
+ *   2B.3 16x16 2D block scaling for weights, 1x16 for activations/gradients;
+ *   2B.4 stochastic rounding on gradients (Dgrad and Wgrad);
+ * and "NVIDIA acelera el preentrenamiento de LLM: NVFP4 en Blackwell junto con
+ * JAX y MaxText", section "Como Funciona Mixed-Precision con NVFP4": GEMMs on
+ * NVFP4 weights and activations with high-precision accumulators.
+ *
+ * Conventions for every call:
+ *  - Pointers marked "device" are CUDA device pointers owned by the caller;
+ *    the library never allocates or frees device memory.
+ *  - Work is enqueued on the caller's stream and never synchronizes the host.
+ *  - Argument errors return immediately, before anything is enqueued.
+ *    NVFP4_ERR_CUDA means a launch failed (cudaGetLastError is left set).
+ *  - BF16 inputs are row-major [R, C] with row pitch ld (elements), finite
+ *    values only; a device pointer must be 16-byte aligned.
+ *  - Per-tensor scale: amax A = max|x| (FP32), S_enc = 2688 / A to encode and
+ *    s_g = A / 2688 to decode (2688 = 6 * 448, the E2M1 and E4M3 maxima); an
+ *    all-zero tensor uses S_enc = s_g = 1.
+ *  - Block scale: d = bamax * S_enc / 6 rounded to nearest E4M3 (saturating at
+ *    448); codes: x * (S_enc / s_b) rounded to E2M1 (nearest-even or
+ *    stochastic), saturating at 6; a zero magnitude is stored as +0.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* nvfp4_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1, /* null pointer where one is required, bad enum */
+  NVFP4_ERR_SHAPE = 2,       /* a dimension breaks the stated divisibility rule */
+  NVFP4_ERR_ALIGN = 3,       /* a pointer or pitch breaks the alignment rule */
+  NVFP4_ERR_UNSUPPORTED = 4, /* a mode/flag combination the method excludes */
+  NVFP4_ERR_DEVICE = 5,      /* current device is not sm_100 */
+  NVFP4_ERR_CUDA = 6,        /* a CUDA launch or driver call failed */
+  NVFP4_ERR_WORKSPACE = 7,   /* workspace missing or smaller than required */
+  NVFP4_ERR_TIMEOUT = 8      /* a kernel gave up on a bounded wait (see nvfp4_read_device_error) */
+} nvfp4_status;
+
+typedef enum {
+  NVFP4_ROW = 1,    /* 1x16 blocks along C; output [R, C/2]                     */
+  NVFP4_COL = 2,    /* 1x16 blocks along R; transposed output [C, R/2]          */
+  NVFP4_ROWCOL = 3, /* both copies from one call (no RHT)                        */
+  NVFP4_2D = 4      /* 16x16 blocks (weights); row and/or column copy            */
+} nvfp4_mode;
+
+typedef enum { NVFP4_OUT_F32 = 0, NVFP4_OUT_BF16 = 1 } nvfp4_out_dtype;
+
+/*
+ * A quantized operand, stored K-major (cols = the contracted dimension K).
+ *   data          device, rows * cols / 2 bytes: codes of row r at
+ *                 data[r * cols/2 ...], element 2i in the low nibble of byte i
+ *                 and element 2i+1 in the high nibble.
+ *   scales        device, nvfp4_scale_bytes(rows, cols) bytes: E4M3 scale of
+ *                 (row r, block c = k / 16) at byte
+ *                   ((r/128) * (Sp/4) + c/4) * 512 + (r%32) * 16 + ((r%128)/32) * 4 + c%4
+ *                 with Sp = pad4(cols/16); rows are padded to a multiple of 128
+ *                 and padding bytes are 0.  This is the 128x4 tile layout the
+ *                 tensor core's block-scaled MMA reads.
+ *   global_scale  device, one float: the decode scale s_g = amax / 2688.
+ */
+typedef struct {
+  void* data;
+  void* scales;
+  float* global_scale;
+  int64_t rows;
+  int64_t cols;
+} nvfp4_tensor;
+
+/* Bytes of packed codes / swizzled scales of a [rows, cols] operand. */
+size_t nvfp4_data_bytes(int64_t rows, int64_t cols);
+size_t nvfp4_scale_bytes(int64_t rows, int64_t cols);
+
+/*
+ * nvfp4_amax -- per-tensor absolute maximum (section 2A, first scaling level).
+ *   x         device BF16 [R, C], pitch ld >= C.
+ *   rht       0: max |x|.  1: max |Q x| where Q = 1/4 * H16 * diag(s) acts on
+ *             every aligned 16-run of rows of each column (section 2B.2; the
+ *             amax of the tensor the Wgrad blocks are taken from).  Needs
+ *             R % 16 == 0, C % 8 == 0, ld % 8 == 0.
+ *   amax_dev  device, one float, overwritten (not accumulated).
+ */
+nvfp4_status nvfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht, float* amax_dev,
+                        nvfp4_stream_t stream);
+
+/*
+ * nvfp4_quantize -- BF16 -> NVFP4 (sections 2A, 2B.2-2B.4).
+ *   x          device BF16 [R, C], pitch ld (ld % 8 == 0).
+ *   mode       NVFP4_ROW: row_out gets rows = R, cols = C (C % 16 == 0).
+ *              NVFP4_COL: col_out gets rows = C, cols = R (R % 16 == 0, C % 4 == 0).
+ *              NVFP4_ROWCOL: both of the above (rht must be 0).
+ *              NVFP4_2D: 16x16 blocks, R % 16 == 0 and C % 16 == 0; row_out
+ *              (rows R, cols C) and/or col_out (rows C, cols R) -- the two
+ *              hold the same codes, transposed, with the 16x16 scale repeated
+ *              over the 16 rows it covers.
+ *   rht        1: apply Q along R before quantizing (COL mode only).
+ *   sr         1: stochastic rounding (ROW, COL, ROWCOL; not 2D).  The word of
+ *              element (r, c) is word ((r*C + c) & 3) of Philox4x32-10 with
+ *              key = seed and counter = ((r*C + c) >> 2, domain, 0), domain 0
+ *              for the row copy and 1 for the column copy; round up iff
+ *              (word >> 8) * 2^-24 < the value's fractional grid position.
+ *   seed       Philox key (used only with sr).
+ *   amax_dev   device float from nvfp4_amax (rht = 1 for an RHT column copy).
+ *   row_out / col_out  caller-filled descriptors (may be NULL when the mode
+ *              does not produce that copy); rows/cols must match the above.
+ *              Their global_scale receives s_g.
+ * Combinations the method excludes return NVFP4_ERR_UNSUPPORTED: RHT on a row
+ * copy or in 2D mode (the RHT is for the Wgrad inputs), SR in 2D mode (SR is
+ * for gradients; weights round to nearest).
+ */
+nvfp4_status nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, nvfp4_mode mode, int rht, int sr,
+                            uint64_t seed, const float* amax_dev, const nvfp4_tensor* row_out,
+                            const nvfp4_tensor* col_out, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_gemm -- block-scaled FP4 GEMM with FP32 accumulation
+ * ("Como Funciona Mixed-Precision con NVFP4"; section 4 of the NVFP4 page):
+ *   D[m, n] = s_gA * s_gB * sum_k dq(A[m, k]) * dq(B[n, k]),  M = A->rows,
+ *   N = B->rows, K = A->cols = B->cols.
+ *   D          device, [M, N] with row pitch ldd; FP32 or BF16 (out_dtype).
+ * Needs K % 64 == 0, N % 16 == 0, ldd % 8 == 0, 16-byte aligned pointers.
+ */
+nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, nvfp4_out_dtype out_dtype,
+                        int64_t ldd, nvfp4_stream_t stream);
+
+/*
+ * Linear layer Y = X W^T with X [T, Cin], W [Cout, Cin] (BF16, contiguous).
+ * Workspace (device, caller-owned, nvfp4_linear_workspace_bytes bytes) holds
+ * the quantized operands; linear_fwd leaves in it what linear_bwd needs.
+ *
+ * nvfp4_linear_fwd: amax(X) -> X row copy (RN); amax(W) -> W 2D (row + column
+ *   copies, RN); Y = gemm(Xq, Wq) in BF16; amax_rht(X) -> X column copy with
+ *   RHT (RN), kept for wgrad.
+ * nvfp4_linear_bwd: amax(dY) -> dY row copy with SR (seed); dX = gemm(dYq, W^T
+ *   column copy) in BF16; amax_rht(dY) -> dY column copy with RHT and SR
+ *   (seed); dW = gemm(dY^T q, X^T q) in FP32.
+ * Needs T, Cin, Cout multiples of 64.
+ */
+size_t nvfp4_linear_workspace_bytes(int64_t T, int64_t Cin, int64_t Cout);
+nvfp4_status nvfp4_linear_fwd(const void* X, const void* W, int64_t T, int64_t Cin, int64_t Cout, void* Y,
+                              void* workspace, size_t workspace_bytes, nvfp4_stream_t stream);
+nvfp4_status nvfp4_linear_bwd(const void* dY, int64_t T, int64_t Cin, int64_t Cout, uint64_t seed, void* dX,
+                              float* dW, void* workspace, size_t workspace_bytes, nvfp4_stream_t stream);
+
+/*
+ * The quantized operands inside a linear workspace (descriptors only; the
+ * memory is the workspace's).  which: 0 X row, 1 W row, 2 W column, 3 X column
+ * (RHT), 4 dY row (SR), 5 dY column (RHT + SR).
+ */
+nvfp4_status nvfp4_linear_workspace_tensor(void* workspace, int64_t T, int64_t Cin, int64_t Cout, int which,
+                                           nvfp4_tensor* out);
+
+/* Device error word written by kernels whose bounded waits ran out (0 = none).
+ * Synchronous; clear != 0 resets it to 0. */
+nvfp4_status nvfp4_read_device_error(unsigned int* code, int clear);
+
+/* Self-test of the bounded wait: enqueues a kernel that waits on a barrier
+ * nothing ever completes; after timeout_us it records error code 5 and ends. */
+nvfp4_status nvfp4_wait_probe(uint32_t timeout_us, nvfp4_stream_t stream);
+
+/* The 16 RHT signs as a bit mask (bit j set: s_j = -1): bits 0..15 of word 0
+ * of Philox4x32-10 with key 0 and counter (0, 0, 2, 0). */
+uint32_t nvfp4_rht_sign_mask(void);
+
+const char* nvfp4_status_string(nvfp4_status status);
+int nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_H */

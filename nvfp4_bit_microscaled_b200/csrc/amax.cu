@@ -1,0 +1,149 @@
+// amax.cu -- per-tensor absolute maximum, plain and after the 16-point RHT.
+//
+// The per-tensor FP32 scale of NVFP4 is derived from the tensor's absolute
+// maximum ("Pretraining Large Language Models with NVFP4", section 2A, first
+// level of the two-level scaling).  For the Wgrad inputs the blocks are taken
+// after a random Hadamard transform (section 2B.2), so their scale comes from
+// max |Q x| over every aligned 16-run along the token dimension.
+//
+// Both kernels are HBM-bound: 2 bytes read per element, one 4-byte result.
+// The result is combined across CTAs with an integer atomicMax on the float's
+// bit pattern (non-negative floats order like their bit patterns).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+
+// Contiguous case: the tensor is a flat array of n elements (n % 8 == 0).
+// Each thread keeps 16-bit magnitude maxima in packed pairs (__vmaxu2), so the
+// inner loop is one AND and one max per two elements.
+__global__ void __launch_bounds__(256) amax_flat_kernel(const uint4* __restrict__ x, int64_t n8,
+                                                          unsigned int* __restrict__ out) {
+  constexpr int U = 8;  // 16-byte loads in flight per thread
+  uint32_t m2 = 0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + (U - 1) * stride < n8; i += U * stride) {
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) v[u] = __ldcs(x + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      m2 = __vmaxu2(m2, v[u].x & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v[u].y & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v[u].z & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v[u].w & 0x7FFF7FFFu);
+    }
+  }
+  for (; i < n8; i += stride) {
+    uint4 v = __ldcs(x + i);
+    m2 = __vmaxu2(m2, absmax_bits8(v));
+  }
+  uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ uint32_t red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = red[0];
+    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) b = max(b, red[w]);
+    if (b) atomicMax(out, b << 16);  // BF16 magnitude bits -> FP32 bit pattern
+  }
+}
+
+// Strided rows (ld != C) or C % 8 != 0: one warp per row, scalar loads.
+__global__ void __launch_bounds__(256) amax_rows_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+                                                          int64_t ld, unsigned int* __restrict__ out) {
+  uint32_t m = 0;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R;
+       r += warps) {
+    const uint16_t* row = x + r * ld;
+    for (int64_t c = lane; c < C; c += 32) m = max(m, static_cast<uint32_t>(row[c] & 0x7FFFu));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if (lane == 0 && m) atomicMax(out, m << 16);
+}
+
+// 16-point fast Walsh-Hadamard butterflies in the fixed order h = 1, 2, 4, 8
+// (natural/Sylvester ordering: out_i = sum_j (-1)^popcount(i & j) in_j).
+__device__ __forceinline__ void fwht16(float (&v)[16]) {
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if ((j & h) == 0) {
+        float a = v[j], b = v[j + h];
+        v[j] = __fadd_rn(a, b);
+        v[j + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+}
+
+// max |Q x| with Q = 1/4 * H16 * diag(s) on each aligned 16-run of rows of
+// every column.  Thread item: one 16-row band x 8 consecutive columns (sixteen
+// 16-byte loads, coalesced across the warp along the row).  The 1/4 is applied
+// after the maximum (an exact power-of-two scale commutes with max).
+__global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+                                                         int64_t ld, uint32_t sign_mask,
+                                                         unsigned int* __restrict__ out) {
+  const int64_t groups = C / 8;
+  const int64_t items = (R / 16) * groups;
+  float m = 0.0f;
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items;
+       it += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t band = it / groups, g = it - band * groups;
+    const uint16_t* base = x + band * 16 * ld + g * 8;
+    uint4 v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __ldcs(reinterpret_cast<const uint4*>(base + i * ld));
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float f[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        uint32_t word = (c < 2) ? v[i].x : (c < 4) ? v[i].y : (c < 6) ? v[i].z : v[i].w;
+        uint32_t bits = (c & 1) ? (word >> 16) : (word & 0xFFFFu);
+        bits ^= ((sign_mask >> i) & 1u) << 15;  // s_i = -1 flips the sign bit
+        f[i] = bf16_bits_to_f32(bits);
+      }
+      fwht16(f);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(f[i]));
+    }
+  }
+  m = __fmul_rn(m, 0.25f);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0 && m > 0.0f) atomicMax(out, __float_as_uint(m));
+}
+
+cudaError_t launch_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht, uint32_t sign_mask,
+                        float* amax_dev, int num_sms, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(amax_dev, 0, sizeof(float), s);
+  if (e != cudaSuccess) return e;
+  if (R == 0 || C == 0) return cudaSuccess;
+  unsigned int* out = reinterpret_cast<unsigned int*>(amax_dev);
+  if (rht) {
+    int64_t items = (R / 16) * (C / 8);
+    int64_t blocks = (items + 255) / 256;
+    int grid = static_cast<int>(blocks < 4LL * num_sms ? blocks : 4LL * num_sms);
+    amax_rht_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), R, C, ld, sign_mask, out);
+  } else if (ld == C && (R * C) % 8 == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
+    int64_t n8 = R * C / 8;
+    int64_t blocks = (n8 + 255) / 256;
+    int grid = static_cast<int>(blocks < 4LL * num_sms ? blocks : 4LL * num_sms);
+    amax_flat_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), n8, out);
+  } else {
+    int64_t blocks = (R + 7) / 8;
+    int grid = static_cast<int>(blocks < 8LL * num_sms ? blocks : 8LL * num_sms);
+    amax_rows_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), R, C, ld, out);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

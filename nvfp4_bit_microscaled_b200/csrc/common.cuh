@@ -1,0 +1,336 @@
+// common.cuh -- device primitives shared by the NVFP4 kernels (sm_100a only).
+//
+// FP4 (E2M1) elements in 16-element blocks with an E4M3 scale per block and an
+// FP32 scale per tensor: "Pretraining Large Language Models with NVFP4",
+// Technische samenvatting, section 2A "Het NVFP4 Formaat".
+//
+// Conversions use the hardware cvt instructions (round-to-nearest-even,
+// saturating to the largest finite value); divisions are IEEE (__fdiv_rn) and
+// every product that must not fuse is spelled __fmul_rn, so the FP32 steps are
+// the same single roundings the method's definition asks for.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#if !defined(__CUDA_ARCH__) || (__CUDA_ARCH__ >= 1000)
+#else
+#error "nvfp4 kernels target sm_100a only"
+#endif
+
+namespace nvfp4 {
+
+// --------------------------------------------------------------------------
+// Error word: kernels that give up on a bounded wait record a code here; the
+// host reads it with nvfp4_read_device_error().  Lives in the library image.
+// --------------------------------------------------------------------------
+extern __device__ unsigned int g_device_error;
+
+enum DeviceError : unsigned int {
+  kErrNone = 0,
+  kErrWaitFull = 1,      // GEMM: MMA issuer waited too long for a loaded stage
+  kErrWaitEmpty = 2,     // GEMM: producer waited too long for a free stage
+  kErrWaitAccFull = 3,   // GEMM: epilogue waited too long for an accumulator
+  kErrWaitAccEmpty = 4,  // GEMM: MMA issuer waited too long for the epilogue
+  kErrWaitProbe = 5,     // wait self-test: nothing ever arrives, by design
+};
+
+__device__ __forceinline__ void record_error(unsigned int code) {
+  atomicCAS(&g_device_error, 0u, code);
+}
+
+// --------------------------------------------------------------------------
+// Small helpers
+// --------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) {
+  return __uint_as_float(b16 << 16);
+}
+
+// |bf16| maximum of eight packed values (a uint4) as 16-bit magnitude bits:
+// clearing the sign bit makes the bit patterns order like the magnitudes.
+__device__ __forceinline__ uint32_t absmax_bits8(uint4 v) {
+  uint32_t a = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+  uint32_t b = __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
+  uint32_t m = __vmaxu2(a, b);
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+// --------------------------------------------------------------------------
+// Format conversions
+// --------------------------------------------------------------------------
+// FP32 -> E4M3, round-to-nearest-even, saturating to 448.
+__device__ __forceinline__ uint32_t f32_to_e4m3(float d) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(d));
+  return r & 0xFFu;
+}
+
+// E4M3 -> FP32 (exact: every E4M3 value is an FP16 value).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+  uint32_t h2;
+  uint16_t in = static_cast<uint16_t>(b & 0xFFu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+
+// Two FP32 values -> one byte of two E2M1 codes: lo in bits 0-3, hi in 4-7.
+// Round-to-nearest-even, saturating to 6.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+      "cvt.u32.u8 %0, t;\n\t}"
+      : "=r"(out)
+      : "f"(hi), "f"(lo));
+  return out;
+}
+
+// A code whose magnitude is zero is stored as +0 (0x0), never as -0 (0x8).
+// Works on eight packed nibbles at once.
+__device__ __forceinline__ uint32_t clear_negative_zero(uint32_t w) {
+  uint32_t mag = w & 0x77777777u;
+  uint32_t nz = (mag | (mag >> 1) | (mag >> 2)) & 0x11111111u;
+  return mag | (w & (nz << 3));
+}
+
+// --------------------------------------------------------------------------
+// Philox4x32-10 (Salmon et al., SC'11), counter-based: four 32-bit words per
+// (counter, key).  Multipliers and Weyl constants are the published ones.
+// --------------------------------------------------------------------------
+struct u32x4 { uint32_t x, y, z, w; };
+
+__host__ __device__ __forceinline__ u32x4 philox4x32_10(u32x4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int round = 0; round < 10; ++round) {
+#if defined(__CUDA_ARCH__)
+    uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+    uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+#else
+    uint64_t p0 = 0xD2511F53ull * c.x, p1 = 0xCD9E8D57ull * c.z;
+    uint32_t hi0 = static_cast<uint32_t>(p0 >> 32), lo0 = static_cast<uint32_t>(p0);
+    uint32_t hi1 = static_cast<uint32_t>(p1 >> 32), lo1 = static_cast<uint32_t>(p1);
+#endif
+    c = u32x4{hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0};
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return c;
+}
+
+// Stochastic rounding counter domains (one Philox stream per use).
+enum : uint32_t { kDomainRowSR = 0, kDomainColSR = 1, kDomainRhtSigns = 2 };
+
+// Words for the four consecutive elements 4g .. 4g+3 (row-major input index).
+__device__ __forceinline__ u32x4 sr_words(uint64_t g, uint32_t domain, uint32_t k0, uint32_t k1) {
+  return philox4x32_10(u32x4{static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), domain, 0u},
+                       k0, k1);
+}
+
+// Stochastic rounding of a scaled value to the E2M1 grid: between the two
+// neighbouring grid magnitudes lo and lo + step, round up iff the 24-bit
+// uniform u = (w >> 8) * 2^-24 is below the fractional position p.  Grid steps
+// are 0.5 on [0,2), 1 on [2,4), 2 on [4,6]; all steps below are exact.
+// ("Pretraining Large Language Models with NVFP4", section 2B.4 and the
+// "De Gok" example: 3.4 goes to 4 with probability 0.4.)
+__device__ __forceinline__ float sr_magnitude(float y, uint32_t w) {
+  float a = fminf(fabsf(y), 6.0f);
+  float step = (a < 2.0f) ? 0.5f : ((a < 4.0f) ? 1.0f : 2.0f);
+  float inv = (a < 2.0f) ? 2.0f : ((a < 4.0f) ? 1.0f : 0.5f);
+  float lo = __fmul_rn(floorf(__fmul_rn(a, inv)), step);
+  float p = __fmul_rn(__fsub_rn(a, lo), inv);
+  float u = __fmul_rn(static_cast<float>(w >> 8), 5.9604644775390625e-08f);  // 2^-24
+  float mag = (u < p) ? __fadd_rn(lo, step) : lo;
+  return copysignf(mag, y);
+}
+
+// --------------------------------------------------------------------------
+// Per-tensor and per-block scales (section 2A, two-level scaling)
+// --------------------------------------------------------------------------
+// Encode scale S_enc = 2688 / amax (2688 = 6 * 448: FP4 max times E4M3 max).
+__device__ __forceinline__ float encode_scale(float amax) {
+  return (amax == 0.0f) ? 1.0f : __fdiv_rn(2688.0f, amax);
+}
+// Decode scale s_g = amax / 2688, the value the GEMM multiplies back.
+__device__ __forceinline__ float decode_scale(float amax) {
+  return (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+}
+
+struct BlockScale {
+  uint32_t sf;   // E4M3 byte
+  float r;       // S_enc / s_b, or 0 when the block's scale decodes to 0
+};
+
+__device__ __forceinline__ BlockScale block_scale(float bamax, float s_enc) {
+  float d = __fdiv_rn(__fmul_rn(bamax, s_enc), 6.0f);
+  BlockScale b;
+  b.sf = f32_to_e4m3(d);
+  float sb = e4m3_to_f32(b.sf);
+  b.r = (sb == 0.0f) ? 0.0f : __fdiv_rn(s_enc, sb);
+  return b;
+}
+
+// --------------------------------------------------------------------------
+// Scale-factor layout: 128x4 tiles of 512 bytes, the block-scale layout the
+// tensor core's block-scaled MMA reads (one tile = 128 rows x 4 scales).
+// --------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t c, int64_t sp) {
+  return ((r >> 7) * (sp >> 2) + (c >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (c & 3);
+}
+
+// --------------------------------------------------------------------------
+// mbarrier, TMA, bulk copy
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+                   smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: gives up after timeout_ns of wall time, records err and returns
+// false.  The caller then leaves its loop (the kernel winds down).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int err,
+                                          uint64_t timeout_ns = 2000000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = globaltimer_ns();
+  for (uint32_t spin = 1;; ++spin) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((spin & 255u) == 0 && globaltimer_ns() - t0 > timeout_ns) {
+      record_error(err);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_t* bar, int32_t x,
+                                            int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const void* tmap) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// --------------------------------------------------------------------------
+// tcgen05 (5th-generation tensor core, tensor memory)
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05): start, leading and stride byte
+// offsets in 16-byte units, descriptor version 1, layout (0 none, 2 = 128B swizzle).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t layout) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= static_cast<uint64_t>(layout & 7u) << 61;
+  return d;
+}
+
+// Copy 32 rows x 16 bytes of shared memory into 4 TMEM columns, replicated over
+// the four 32-lane sub-partitions (the layout the block-scaled MMA expects for
+// a 128x4 scale tile).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T with per-16-element E4M3 scales from TMEM.
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t"
+      "}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on an mbarrier once every tcgen05 operation issued so far by this
+// thread has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+}  // namespace nvfp4

@@ -1,0 +1,329 @@
+// gemm.cu -- block-scaled FP4 x FP4 -> FP32 GEMM on the 5th-generation tensor core.
+//
+//   D[m, n] = (s_gA * s_gB) * sum_k e2m1(A[m,k]) e4m3(sA[m,k/16]) e2m1(B[n,k]) e4m3(sB[n,k/16])
+//
+// NVFP4 GEMMs take FP4 weights and activations and keep the accumulator in
+// high precision ("NVIDIA acelera el preentrenamiento de LLM: NVFP4 en
+// Blackwell junto con JAX y MaxText", section "Como Funciona Mixed-Precision
+// con NVFP4"); Blackwell tensor cores run NVFP4 natively ("Pretraining Large
+// Language Models with NVFP4", section 4).  The same kernel serves fprop
+// (Y = X W^T), dgrad (dX = dY W) and wgrad (dW = dY^T X): every operand is
+// stored K-major (the contracted dimension contiguous).
+//
+// Design (persistent, warp-specialised, one CTA per SM):
+//   warp 0  TMA producer: A tile 128 x 256 and B tile 256 x 256 (packed FP4,
+//           128-byte swizzle) plus their 128x4 scale tiles (1-D bulk copies)
+//           into a 4-stage shared-memory ring guarded by mbarriers;
+//   warp 1  MMA issuer: copies the stage's scales to tensor memory
+//           (tcgen05.cp) and issues four tcgen05.mma kind::mxf4nvf4 (K = 64
+//           each, 16-element E4M3 block scales) into a 128 x 256 FP32
+//           accumulator in tensor memory; tcgen05.commit frees the stage;
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator, x alpha, store FP32
+//           or BF16; then hand the accumulator back to the MMA issuer.
+// Every mbarrier wait is bounded; on a timeout the kernel records an error
+// word, lets in-flight copies and MMAs land, frees tensor memory and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+
+__device__ unsigned int g_device_error = 0;
+
+namespace {
+
+constexpr int BM = 128;              // rows of A per tile
+constexpr int BN = 256;              // rows of B per tile (columns of D)
+constexpr int BK_BYTES = 128;        // packed K bytes per stage (256 FP4 values)
+constexpr int KB_PER_STAGE = 4;      // 64-element MMA steps per stage
+constexpr int STAGES = 4;
+constexpr uint32_t A_BYTES = BM * BK_BYTES;                  // 16 KiB
+constexpr uint32_t B_BYTES = BN * BK_BYTES;                  // 32 KiB
+constexpr uint32_t SFA_BYTES = KB_PER_STAGE * 512;           // 2 KiB
+constexpr uint32_t SFB_BYTES = 2 * KB_PER_STAGE * 512;       // 4 KiB
+constexpr uint32_t OFF_A = 0;
+constexpr uint32_t OFF_B = OFF_A + STAGES * A_BYTES;
+constexpr uint32_t OFF_SFA = OFF_B + STAGES * B_BYTES;
+constexpr uint32_t OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+constexpr uint32_t OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;        // + barriers + alignment slack
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 256 + 16;
+constexpr int GROUP_M = 16;                                  // tile raster: 16 M-tiles share B tiles in L2
+
+// Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1), K-major,
+// UE4M3 scales, dense K = 64, M = 128.
+__host__ __device__ constexpr uint32_t make_idesc(int n) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (0u << 23) |
+         (static_cast<uint32_t>(BM >> 4) << 24);
+}
+
+struct TileCoord { int m, n; };
+
+__device__ __forceinline__ TileCoord tile_coord(int t, int num_m, int num_n) {
+  const int per_group = GROUP_M * num_n;
+  const int grp = t / per_group;
+  const int first_m = grp * GROUP_M;
+  const int gsize = min(num_m - first_m, GROUP_M);
+  const int within = t - grp * per_group;
+  return TileCoord{first_m + within % gsize, within / gsize};
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb, const float* __restrict__ gsa,
+                 const float* __restrict__ gsb, int M, int N, int K, void* __restrict__ D, int out_bf16,
+                 int64_t ldd) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* mma_done = acc_empty + 1;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(mma_done + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int katoms = (K + 63) / 64;          // 128x4 scale tiles along K (= pad4(K/16) / 4)
+  const int num_kt = (K + 255) / 256;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) tmem_alloc(const_cast<uint32_t*>(tmem_slot), TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_parity[STAGES];
+    bool issued[STAGES];
+    for (int s = 0; s < STAGES; ++s) issued[s] = false, issued_parity[s] = 0;
+    for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+      const TileCoord tc = tile_coord(t, num_m, num_n);
+      const bool second_half = tc.n * BN + 128 < N;
+      for (int kt = 0; kt < num_kt; ++kt) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, kErrWaitEmpty)) { *abort_flag = 1; break; }
+        const int nkb = min(KB_PER_STAGE, katoms - kt * KB_PER_STAGE);
+        const uint32_t sf_bytes = static_cast<uint32_t>(nkb) * 512u;
+        const uint32_t bytes = A_BYTES + B_BYTES + sf_bytes * (second_half ? 3u : 2u);
+        mbar_arrive_expect_tx(&full[stage], bytes);
+        tma_load_2d(smem + OFF_A + stage * A_BYTES, &tmA, &full[stage], kt * BK_BYTES, tc.m * BM);
+        tma_load_2d(smem + OFF_B + stage * B_BYTES, &tmB, &full[stage], kt * BK_BYTES, tc.n * BN);
+        bulk_load(smem + OFF_SFA + stage * SFA_BYTES,
+                  sfa + (static_cast<int64_t>(tc.m) * katoms + kt * KB_PER_STAGE) * 512, sf_bytes, &full[stage]);
+        bulk_load(smem + OFF_SFB + stage * SFB_BYTES,
+                  sfb + (static_cast<int64_t>(2 * tc.n) * katoms + kt * KB_PER_STAGE) * 512, sf_bytes,
+                  &full[stage]);
+        if (second_half)
+          bulk_load(smem + OFF_SFB + stage * SFB_BYTES + KB_PER_STAGE * 512,
+                    sfb + (static_cast<int64_t>(2 * tc.n + 1) * katoms + kt * KB_PER_STAGE) * 512, sf_bytes,
+                    &full[stage]);
+        issued[stage] = true;
+        issued_parity[stage] = phase;
+        if (++stage == STAGES) stage = 0, phase ^= 1u;
+      }
+    }
+    // Let every copy this thread started land before the CTA can exit.
+    for (int s = 0; s < STAGES; ++s)
+      if (issued[s]) mbar_wait(&full[s], issued_parity[s], kErrWaitFull);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    int stage = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    const uint32_t a_base = smem_u32(smem + OFF_A), b_base = smem_u32(smem + OFF_B);
+    const uint32_t sfa_base = smem_u32(smem + OFF_SFA), sfb_base = smem_u32(smem + OFF_SFB);
+    for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+      const TileCoord tc = tile_coord(t, num_m, num_n);
+      const bool second_half = tc.n * BN + 128 < N;
+      const uint32_t idesc = make_idesc(second_half ? 256 : 128);
+      if (!mbar_wait(acc_empty, acc_phase ^ 1u, kErrWaitAccEmpty)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      bool ok = true;
+      for (int kt = 0; kt < num_kt; ++kt) {
+        if (!mbar_wait(&full[stage], phase, kErrWaitFull)) { ok = false; break; }
+        tc_fence_after();
+        const int nkb = min(KB_PER_STAGE, katoms - kt * KB_PER_STAGE);
+        const uint32_t sfa_s = sfa_base + stage * SFA_BYTES, sfb_s = sfb_base + stage * SFB_BYTES;
+        for (int kb = 0; kb < nkb; ++kb) {
+          tmem_cp_32x128b_x4(tmem + SFA_COL + 4 * kb, smem_desc(sfa_s + 512 * kb, 16, 128, 0));
+          tmem_cp_32x128b_x4(tmem + SFB_COL + 8 * kb, smem_desc(sfb_s + 512 * kb, 16, 128, 0));
+          if (second_half)
+            tmem_cp_32x128b_x4(tmem + SFB_COL + 8 * kb + 4,
+                               smem_desc(sfb_s + KB_PER_STAGE * 512 + 512 * kb, 16, 128, 0));
+        }
+        const uint64_t adesc = smem_desc(a_base + stage * A_BYTES, 16, 1024, 2);
+        const uint64_t bdesc = smem_desc(b_base + stage * B_BYTES, 16, 1024, 2);
+        for (int kb = 0; kb < nkb; ++kb) {
+          // +32 bytes along K inside the 128-byte swizzle row = +2 in the 16-byte address field
+          mma_nvf4(tmem + ACC_COL, adesc + 2 * kb, bdesc + 2 * kb, idesc, tmem + SFA_COL + 4 * kb,
+                   tmem + SFB_COL + 8 * kb, (kt | kb) != 0);
+        }
+        tc_commit(&empty[stage]);
+        if (++stage == STAGES) stage = 0, phase ^= 1u;
+      }
+      if (!ok) { *abort_flag = 1; break; }
+      tc_commit(acc_full);
+      acc_phase ^= 1u;
+    }
+    // Let every MMA this thread issued finish before tensor memory is freed.
+    tc_commit(mma_done);
+    mbar_wait(mma_done, 0, kErrWaitAccFull);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // tensor-memory lanes this warp may read
+    const float alpha = __fmul_rn(__ldg(gsa), __ldg(gsb));
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+      const TileCoord tc = tile_coord(t, num_m, num_n);
+      if (!mbar_wait(acc_full, acc_phase, kErrWaitAccFull)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      const int row = tc.m * BM + quarter * 32 + lane;
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        const int col0 = tc.n * BN + ch * 32;
+        if (col0 >= N) break;
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ACC_COL + ch * 32, r);
+        tmem_ld_wait();
+        if (row < M) {
+          const int ncols = min(32, N - col0);
+          if (out_bf16) {
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(D) + static_cast<int64_t>(row) * ldd + col0;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (v * 8 < ncols) {
+                uint32_t p[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[v * 8 + 2 * e]), alpha),
+                                                           __fmul_rn(__uint_as_float(r[v * 8 + 2 * e + 1]), alpha));
+                  p[e] = *reinterpret_cast<uint32_t*>(&h);
+                }
+                reinterpret_cast<uint4*>(dst)[v] = make_uint4(p[0], p[1], p[2], p[3]);
+              }
+            }
+          } else {
+            float* dst = static_cast<float*>(D) + static_cast<int64_t>(row) * ldd + col0;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              if (v * 4 < ncols) {
+                reinterpret_cast<float4*>(dst)[v] =
+                    make_float4(__fmul_rn(__uint_as_float(r[4 * v + 0]), alpha),
+                                __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
+                                __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha),
+                                __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      acc_phase ^= 1u;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// K-major packed FP4 operand [rows, K/2] bytes; box = 128 bytes x box_rows,
+// 128-byte swizzle (the canonical K-major layout the MMA descriptors name).
+bool make_operand_map(CUtensorMap* tm, const void* data, int64_t rows, int64_t K, int box_rows) {
+  auto encode = get_encode_fn();
+  if (!encode) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK_BYTES), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(data), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a_gs, const void* b_data,
+                        const void* b_scales, const float* b_gs, int64_t M, int64_t N, int64_t K, void* D,
+                        int out_bf16, int64_t ldd, int num_sms, cudaStream_t s) {
+  CUtensorMap tmA, tmB;
+  if (!make_operand_map(&tmA, a_data, M, K, BM) || !make_operand_map(&tmB, b_data, N, K, BN))
+    return cudaErrorInvalidValue;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(SMEM_BYTES));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+  gemm_nvf4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(
+      tmA, tmB, static_cast<const uint8_t*>(a_scales), static_cast<const uint8_t*>(b_scales), a_gs, b_gs,
+      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), D, out_bf16, ldd);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Bounded-wait self-test: the barrier below never completes (nothing arrives),
+// so the wait must give up after timeout_us and record kErrWaitProbe.
+// ---------------------------------------------------------------------------
+__global__ void wait_probe_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, kErrWaitProbe, timeout_ns);
+}
+
+cudaError_t launch_wait_probe(uint32_t timeout_us, cudaStream_t s) {
+  wait_probe_kernel<<<1, 32, 0, s>>>(static_cast<uint64_t>(timeout_us) * 1000ull);
+  return cudaGetLastError();
+}
+
+cudaError_t read_device_error(unsigned int* out, int clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_device_error, sizeof(unsigned int));
+  if (e != cudaSuccess || !clear) return e;
+  const unsigned int zero = 0;
+  return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace nvfp4

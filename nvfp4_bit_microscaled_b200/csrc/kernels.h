@@ -1,0 +1,41 @@
+// kernels.h -- internal launchers behind the C ABI (not part of the public header).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nvfp4 {
+
+cudaError_t launch_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht, uint32_t sign_mask,
+                        float* amax_dev, int num_sms, cudaStream_t s);
+
+// Row-wise 1x16 quantization: data [R, C/2], scales in the 128x4-tile layout
+// with sp = pad4(C/16) scale columns.
+cudaError_t launch_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, const float* amax_dev, int sr,
+                             uint64_t seed, void* data, void* scales, float* gs_out, int num_sms,
+                             cudaStream_t s);
+
+// Column-wise 1x16 quantization along R, optional RHT and SR; transposed
+// output data [C, R/2], scales with sp = pad4(R/16).
+cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, const float* amax_dev, int rht,
+                             uint32_t sign_mask, int sr, uint64_t seed, void* data, void* scales,
+                             float* gs_out, int num_sms, cudaStream_t s);
+
+// 2D 16x16 quantization of W [N, K]: row copy [N, K/2] and/or column copy [K, N/2].
+cudaError_t launch_quant_2d(const void* w, int64_t N, int64_t K, int64_t ld, const float* amax_dev,
+                            void* row_data, void* row_scales, float* row_gs, void* col_data, void* col_scales,
+                            float* col_gs, int num_sms, cudaStream_t s);
+
+// Zero the padding of a scale matrix (rows >= R or scale columns >= S).
+cudaError_t launch_sf_pad_zero(void* scales, int64_t R, int64_t S, cudaStream_t s);
+
+// Block-scaled FP4 GEMM: D[M,N] = sgA * sgB * sum_k A[m,k] B[n,k].
+cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a_gs, const void* b_data,
+                        const void* b_scales, const float* b_gs, int64_t M, int64_t N, int64_t K, void* D,
+                        int out_bf16, int64_t ldd, int num_sms, cudaStream_t s);
+
+// Bounded-wait self-test: a kernel waits on an mbarrier nobody arrives on.
+cudaError_t launch_wait_probe(uint32_t timeout_us, cudaStream_t s);
+
+cudaError_t read_device_error(unsigned int* out, int clear);
+
+}  // namespace nvfp4

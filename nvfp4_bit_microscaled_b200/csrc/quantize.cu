@@ -1,0 +1,420 @@
+// quantize.cu -- BF16 -> NVFP4 (packed E2M1 codes + E4M3 block scales).
+//
+// "Pretraining Large Language Models with NVFP4", Technische samenvatting:
+//   2A    16-element blocks, one E4M3 scale per block, one FP32 scale per tensor;
+//   2B.2  16x16 random Hadamard transform on the Wgrad inputs (column path);
+//   2B.3  1x16 blocks for activations and gradients, 16x16 blocks for weights
+//         so that W and W^T quantize to the same codes;
+//   2B.4  stochastic rounding on gradients (Dgrad and Wgrad inputs).
+//
+// Per block: bamax -> d = bamax * S_enc / 6 -> E4M3 scale s_b (round to
+// nearest) -> r = S_enc / s_b -> y = x * r -> E2M1 code (RN or SR).  All of it
+// is FP32 with single IEEE roundings in that order.
+//
+// The kernels are HBM-bound (2 bytes read, 0.5625 bytes written per element
+// and copy); each thread streams whole 16-element blocks with 8- or 16-byte
+// loads that are coalesced across the warp.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+
+namespace {
+
+// Eight scaled values -> eight nibbles, element 0 in the low nibble.
+__device__ __forceinline__ uint32_t pack8(const float* y) {
+  uint32_t w = f32x2_to_e2m1x2(y[0], y[1]) | (f32x2_to_e2m1x2(y[2], y[3]) << 8) |
+               (f32x2_to_e2m1x2(y[4], y[5]) << 16) | (f32x2_to_e2m1x2(y[6], y[7]) << 24);
+  return clear_negative_zero(w);
+}
+
+__device__ __forceinline__ void unpack8(uint4 v, float* f) {
+  f[0] = bf16_bits_to_f32(v.x & 0xFFFFu); f[1] = bf16_bits_to_f32(v.x >> 16);
+  f[2] = bf16_bits_to_f32(v.y & 0xFFFFu); f[3] = bf16_bits_to_f32(v.y >> 16);
+  f[4] = bf16_bits_to_f32(v.z & 0xFFFFu); f[5] = bf16_bits_to_f32(v.z >> 16);
+  f[6] = bf16_bits_to_f32(v.w & 0xFFFFu); f[7] = bf16_bits_to_f32(v.w >> 16);
+}
+
+__device__ __forceinline__ void fwht16(float (&v)[16]) {
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if ((j & h) == 0) {
+        float a = v[j], b = v[j + h];
+        v[j] = __fadd_rn(a, b);
+        v[j + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Row-wise 1x16 (activations X for fprop, gradients dY for dgrad with SR).
+// Warp item: one row segment of 32 blocks (512 elements); lane = block.
+// Scale bytes of lanes 4j..4j+3 form one 32-bit word of the 128x4 tile layout.
+// ---------------------------------------------------------------------------
+template <bool SR>
+__global__ void __launch_bounds__(256) quant_row_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+                                                          int64_t ld, const float* __restrict__ amax_dev,
+                                                          uint32_t k0, uint32_t k1, uint8_t* __restrict__ data,
+                                                          uint8_t* __restrict__ sf, int64_t sp,
+                                                          float* __restrict__ gs_out) {
+  constexpr int U = 2;  // items in flight per warp
+  const float amax = __ldg(amax_dev);
+  const float s_enc = encode_scale(amax);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && gs_out) *gs_out = decode_scale(amax);
+  const int lane = threadIdx.x & 31;
+  const int64_t S = C >> 4;
+  const int64_t nseg = (S + 31) >> 5;
+  const int64_t items = R * nseg;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t half_c = C >> 1;
+
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); base < items;
+       base += U * nwarps) {
+    uint4 v[U][2];
+    int64_t rr[U], bb[U];
+    bool ok[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t it = base + u * nwarps;
+      const int64_t r = it / nseg;
+      const int64_t b = (it - r * nseg) * 32 + lane;
+      rr[u] = r;
+      bb[u] = b;
+      ok[u] = (it < items) && (b < S);
+      v[u][0] = v[u][1] = make_uint4(0, 0, 0, 0);
+      if (ok[u]) {
+        const uint4* src = reinterpret_cast<const uint4*>(x + r * ld + b * 16);
+        v[u][0] = __ldcs(src);
+        v[u][1] = __ldcs(src + 1);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (base + u * nwarps >= items) break;  // warp-uniform
+      const uint32_t mb = max(absmax_bits8(v[u][0]), absmax_bits8(v[u][1]));
+      const BlockScale bs = block_scale(bf16_bits_to_f32(mb), s_enc);
+      float y[16];
+      unpack8(v[u][0], y);
+      unpack8(v[u][1], y + 8);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(y[i], bs.r);
+      if (SR) {
+        const uint64_t g = static_cast<uint64_t>(rr[u] * C + bb[u] * 16) >> 2;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const u32x4 w = sr_words(g + q, kDomainRowSR, k0, k1);
+          y[4 * q + 0] = sr_magnitude(y[4 * q + 0], w.x);
+          y[4 * q + 1] = sr_magnitude(y[4 * q + 1], w.y);
+          y[4 * q + 2] = sr_magnitude(y[4 * q + 2], w.z);
+          y[4 * q + 3] = sr_magnitude(y[4 * q + 3], w.w);
+        }
+      }
+      const uint32_t w0 = pack8(y), w1 = pack8(y + 8);
+      if (ok[u]) *reinterpret_cast<uint2*>(data + rr[u] * half_c + bb[u] * 8) = make_uint2(w0, w1);
+      uint32_t word = ok[u] ? (bs.sf << (8 * (lane & 3))) : 0u;
+      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+      if ((lane & 3) == 0 && ok[u]) *reinterpret_cast<uint32_t*>(sf + sf_offset(rr[u], bb[u], sp)) = word;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Column-wise 1x16 along R (the tokens: K of the Wgrad GEMM), transposed
+// output.  Thread item: 64 tokens x 4 channels.  Each 16-token block of a
+// channel is optionally rotated by Q = 1/4 H16 diag(s) before it is scaled.
+// Loads: 16 rows x 8 bytes per block (coalesced along the row across the
+// warp); stores: 32 bytes of codes and one 4-byte scale word per channel.
+// SR word for element (t, c): Philox counter (t*C + c) >> 2, so one call
+// serves the four channels of a row.
+// ---------------------------------------------------------------------------
+template <bool RHT, bool SR>
+__global__ void __launch_bounds__(256) quant_col_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+                                                          int64_t ld, const float* __restrict__ amax_dev,
+                                                          uint32_t sign_mask, uint32_t k0, uint32_t k1,
+                                                          uint8_t* __restrict__ data, uint8_t* __restrict__ sf,
+                                                          int64_t sp, float* __restrict__ gs_out) {
+  const float amax = __ldg(amax_dev);
+  const float s_enc = encode_scale(amax);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && gs_out) *gs_out = decode_scale(amax);
+  const int64_t S = R >> 4;
+  const int64_t nq = (S + 3) >> 2;
+  const int64_t ng = C >> 2;
+  const int64_t items = nq * ng;
+  const int64_t half_r = R >> 1;
+  const bool vec_store = (R & 31) == 0;
+
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items;
+       it += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t q = it / ng, g = it - q * ng;
+    const int64_t c0 = g * 4, t0 = q * 64;
+    const int nb = static_cast<int>((S - 4 * q) < 4 ? (S - 4 * q) : 4);
+    uint32_t lo[4][4], hi[4][4];  // [channel][block] codes (8 nibbles each half)
+    uint32_t sfw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int tb = 0; tb < 4; ++tb) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) lo[c][tb] = hi[c][tb] = 0u;
+      if (tb >= nb) continue;
+      const int64_t tbase = t0 + 16 * tb;
+      float v[4][16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint2 raw = __ldcs(reinterpret_cast<const uint2*>(x + (tbase + i) * ld + c0));
+        const uint32_t flip = RHT ? (((sign_mask >> i) & 1u) * 0x80008000u) : 0u;
+        const uint32_t a = raw.x ^ flip, b = raw.y ^ flip;
+        v[0][i] = bf16_bits_to_f32(a & 0xFFFFu);
+        v[1][i] = bf16_bits_to_f32(a >> 16);
+        v[2][i] = bf16_bits_to_f32(b & 0xFFFFu);
+        v[3][i] = bf16_bits_to_f32(b >> 16);
+      }
+      float r[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (RHT) {
+          fwht16(v[c]);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[c][i] = __fmul_rn(v[c][i], 0.25f);
+        }
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[c][i]));
+        const BlockScale bs = block_scale(m, s_enc);
+        r[c] = bs.r;
+        sfw[c] |= bs.sf << (8 * tb);
+      }
+#pragma unroll
+      for (int i = 0; i < 16; i += 2) {
+        float y0[4], y1[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          y0[c] = __fmul_rn(v[c][i], r[c]);
+          y1[c] = __fmul_rn(v[c][i + 1], r[c]);
+        }
+        if (SR) {
+          const u32x4 wa = sr_words(static_cast<uint64_t>((tbase + i) * C + c0) >> 2, kDomainColSR, k0, k1);
+          const u32x4 wb = sr_words(static_cast<uint64_t>((tbase + i + 1) * C + c0) >> 2, kDomainColSR, k0, k1);
+          y0[0] = sr_magnitude(y0[0], wa.x); y0[1] = sr_magnitude(y0[1], wa.y);
+          y0[2] = sr_magnitude(y0[2], wa.z); y0[3] = sr_magnitude(y0[3], wa.w);
+          y1[0] = sr_magnitude(y1[0], wb.x); y1[1] = sr_magnitude(y1[1], wb.y);
+          y1[2] = sr_magnitude(y1[2], wb.z); y1[3] = sr_magnitude(y1[3], wb.w);
+        }
+        const int sh = 8 * ((i >> 1) & 3);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t byte = f32x2_to_e2m1x2(y0[c], y1[c]) << sh;
+          if (i < 8) lo[c][tb] |= byte; else hi[c][tb] |= byte;
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        lo[c][tb] = clear_negative_zero(lo[c][tb]);
+        hi[c][tb] = clear_negative_zero(hi[c][tb]);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint8_t* dst = data + (c0 + c) * half_r + t0 / 2;
+      if (nb == 4 && vec_store) {
+        reinterpret_cast<uint4*>(dst)[0] = make_uint4(lo[c][0], hi[c][0], lo[c][1], hi[c][1]);
+        reinterpret_cast<uint4*>(dst)[1] = make_uint4(lo[c][2], hi[c][2], lo[c][3], hi[c][3]);
+      } else {
+#pragma unroll
+        for (int tb = 0; tb < 4; ++tb)
+          if (tb < nb) reinterpret_cast<uint2*>(dst)[tb] = make_uint2(lo[c][tb], hi[c][tb]);
+      }
+      *reinterpret_cast<uint32_t*>(sf + sf_offset(c0 + c, 4 * q, sp)) = sfw[c];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2D 16x16 (weights).  CTA tile: 64 rows (4 bands of 16, one per warp) x 512
+// columns (32 tiles, one per lane).  Pass 1 reads the tile for its maximum,
+// pass 2 re-reads it (L1-resident) and emits the codes twice: row copy
+// [N, K/2] and column copy [K, N/2] with the nibbles transposed in registers.
+// Scale words of both copies are assembled in shared memory.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) quant_2d_kernel(const uint16_t* __restrict__ w, int64_t N, int64_t K,
+                                                         int64_t ld, const float* __restrict__ amax_dev,
+                                                         uint8_t* __restrict__ row_data, uint8_t* __restrict__ row_sf,
+                                                         int64_t row_sp, float* __restrict__ row_gs,
+                                                         uint8_t* __restrict__ col_data, uint8_t* __restrict__ col_sf,
+                                                         int64_t col_sp, float* __restrict__ col_gs) {
+  __shared__ uint32_t tsf[4][32];
+  const float amax = __ldg(amax_dev);
+  const float s_enc = encode_scale(amax);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (row_gs) *row_gs = decode_scale(amax);
+    if (col_gs) *col_gs = decode_scale(amax);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t TN = N >> 4, TK = K >> 4;
+  const int64_t ctas_k = (TK + 31) >> 5, ctas_n = (TN + 3) >> 2;
+  const int64_t half_k = K >> 1, half_n = N >> 1;
+
+  for (int64_t ci = blockIdx.x; ci < ctas_n * ctas_k; ci += gridDim.x) {
+    const int64_t cn = ci / ctas_k, ck = ci - cn * ctas_k;
+    const int64_t bn = cn * 4 + warp, bk = ck * 32 + lane;
+    const bool ok = (bn < TN) && (bk < TK);
+    const uint16_t* tile = w + bn * 16 * ld + bk * 16;
+    uint32_t mb = 0;
+    if (ok) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint4* src = reinterpret_cast<const uint4*>(tile + i * ld);
+        mb = max(mb, max(absmax_bits8(__ldg(src)), absmax_bits8(__ldg(src + 1))));
+      }
+    }
+    const BlockScale bs = block_scale(bf16_bits_to_f32(mb), s_enc);
+    tsf[warp][lane] = ok ? bs.sf : 0u;
+    if (ok) {
+      uint32_t colw[16][2];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) colw[j][0] = colw[j][1] = 0u;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint4* src = reinterpret_cast<const uint4*>(tile + i * ld);
+        float y[16];
+        unpack8(__ldg(src), y);
+        unpack8(__ldg(src + 1), y + 8);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) y[j] = __fmul_rn(y[j], bs.r);
+        const uint32_t w0 = pack8(y), w1 = pack8(y + 8);
+        if (row_data) *reinterpret_cast<uint2*>(row_data + (bn * 16 + i) * half_k + bk * 8) = make_uint2(w0, w1);
+        // column copy: code (i, j) becomes nibble i of column row j
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint32_t nib = ((j < 8 ? w0 : w1) >> (4 * (j & 7))) & 0xFu;
+          colw[j][i >> 3] |= nib << (4 * (i & 7));
+        }
+      }
+      if (col_data) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          *reinterpret_cast<uint2*>(col_data + (bk * 16 + j) * half_n + bn * 8) = make_uint2(colw[j][0], colw[j][1]);
+      }
+    }
+    __syncthreads();
+    // row copy scales: 64 rows x 8 words (4 tiles each)
+    if (row_sf) {
+      for (int e = threadIdx.x; e < 64 * 8; e += blockDim.x) {
+        const int band = e >> 7, i = (e >> 3) & 15, wq = e & 7;
+        const int64_t n = (cn * 4 + band) * 16 + i, kb = ck * 32 + wq * 4;
+        if (n < N && kb < TK) {
+          const uint32_t word = tsf[band][4 * wq] | (tsf[band][4 * wq + 1] << 8) | (tsf[band][4 * wq + 2] << 16) |
+                                (tsf[band][4 * wq + 3] << 24);
+          *reinterpret_cast<uint32_t*>(row_sf + sf_offset(n, kb, row_sp)) = word;
+        }
+      }
+    }
+    // column copy scales: 512 rows (k) x one word (4 bands)
+    if (col_sf) {
+      for (int e = threadIdx.x; e < 512; e += blockDim.x) {
+        const int t = e >> 4, j = e & 15;
+        const int64_t k = (ck * 32 + t) * 16 + j;
+        if (ck * 32 + t < TK) {
+          const uint32_t word = tsf[0][t] | (tsf[1][t] << 8) | (tsf[2][t] << 16) | (tsf[3][t] << 24);
+          *reinterpret_cast<uint32_t*>(col_sf + sf_offset(k, cn * 4, col_sp)) = word;
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Padding of the scale matrix (rows R..pad128(R), scale columns S..pad4(S)).
+// ---------------------------------------------------------------------------
+__global__ void sf_pad_zero_kernel(uint8_t* __restrict__ sf, int64_t R, int64_t S, int64_t Rp, int64_t Sp) {
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < Rp * Sp;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = e / Sp, c = e - r * Sp;
+    if (r >= R || c >= S) sf[sf_offset(r, c, Sp)] = 0;
+  }
+}
+
+cudaError_t launch_sf_pad_zero(void* scales, int64_t R, int64_t S, cudaStream_t s) {
+  const int64_t Rp = (R + 127) / 128 * 128, Sp = (S + 3) / 4 * 4;
+  if (Rp == R && Sp == S) return cudaSuccess;
+  const int64_t n = Rp * Sp;
+  const int grid = static_cast<int>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
+  sf_pad_zero_kernel<<<grid, 256, 0, s>>>(static_cast<uint8_t*>(scales), R, S, Rp, Sp);
+  return cudaGetLastError();
+}
+
+static inline int grid_for(int64_t work_units, int per_block, int num_sms, int waves) {
+  int64_t blocks = (work_units + per_block - 1) / per_block;
+  int64_t cap = static_cast<int64_t>(num_sms) * waves;
+  if (blocks > cap) blocks = cap;
+  return static_cast<int>(blocks < 1 ? 1 : blocks);
+}
+
+cudaError_t launch_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, const float* amax_dev, int sr,
+                             uint64_t seed, void* data, void* scales, float* gs_out, int num_sms,
+                             cudaStream_t s) {
+  const int64_t S = C / 16, sp = (S + 3) / 4 * 4;
+  const int64_t warp_items = R * ((S + 31) / 32);
+  const int grid = grid_for(warp_items, 8 * 2, num_sms, 8);
+  const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
+  auto* xs = static_cast<const uint16_t*>(x);
+  auto* d = static_cast<uint8_t*>(data);
+  auto* f = static_cast<uint8_t*>(scales);
+  if (sr)
+    quant_row_kernel<true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+  else
+    quant_row_kernel<false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_sf_pad_zero(scales, R, S, s);
+}
+
+cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, const float* amax_dev, int rht,
+                             uint32_t sign_mask, int sr, uint64_t seed, void* data, void* scales,
+                             float* gs_out, int num_sms, cudaStream_t s) {
+  const int64_t S = R / 16, sp = (S + 3) / 4 * 4;
+  const int64_t items = ((S + 3) / 4) * (C / 4);
+  const int grid = grid_for(items, 256, num_sms, 8);
+  const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
+  auto* xs = static_cast<const uint16_t*>(x);
+  auto* d = static_cast<uint8_t*>(data);
+  auto* f = static_cast<uint8_t*>(scales);
+  if (rht && sr)
+    quant_col_kernel<true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+  else if (rht)
+    quant_col_kernel<true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+  else if (sr)
+    quant_col_kernel<false, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+  else
+    quant_col_kernel<false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_sf_pad_zero(scales, C, S, s);
+}
+
+cudaError_t launch_quant_2d(const void* w, int64_t N, int64_t K, int64_t ld, const float* amax_dev,
+                            void* row_data, void* row_scales, float* row_gs, void* col_data, void* col_scales,
+                            float* col_gs, int num_sms, cudaStream_t s) {
+  const int64_t TN = N / 16, TK = K / 16;
+  const int64_t ctas = ((TN + 3) / 4) * ((TK + 31) / 32);
+  const int grid = grid_for(ctas, 1, num_sms, 12);
+  quant_2d_kernel<<<grid, 128, 0, s>>>(static_cast<const uint16_t*>(w), N, K, ld, amax_dev,
+                                       static_cast<uint8_t*>(row_data), static_cast<uint8_t*>(row_scales),
+                                       (TK + 3) / 4 * 4, row_gs, static_cast<uint8_t*>(col_data),
+                                       static_cast<uint8_t*>(col_scales), (TN + 3) / 4 * 4, col_gs);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (row_scales) {
+    e = launch_sf_pad_zero(row_scales, N, TK, s);
+    if (e != cudaSuccess) return e;
+  }
+  if (col_scales) e = launch_sf_pad_zero(col_scales, K, TN, s);
+  return e;
+}
+
+}  // namespace nvfp4
