@@ -1,0 +1,514 @@
+"""Benchmark of the NVFP4 quantized linear layer on B200.
+
+One step = one full pass of the hot path over one batch: forward (amax, X
+row quantize, W 2D quantize, fprop GEMM, X column quantize with RHT) and
+backward (dY amax, dY row quantize with SR, dgrad GEMM, dY RHT amax, dY column
+quantize with RHT + SR, wgrad GEMM), on the "full" workload: T = 16384 tokens,
+hidden 5120 -> FFN 20480 (a 12B hybrid Mamba-Transformer's FFN up-projection),
+seeded synthetic BF16 inputs resident in HBM.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun (N > 1) every rank runs its own batch (weak scaling, no
+collective on the data path); rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (the plain C reference) on the host cores
+on a bounded sample of the same workload.
+"""
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from nvfp4_bit_microscaled_b200 import api, synth  # noqa: E402
+
+METRIC = "NVFP4 GEMM TFLOPS (% dense FP4 peak); quantize GB/s (% HBM peak)"
+WORKLOAD = dict(name="full", T=16384, Cin=5120, Cout=20480, seed=2, sr_seed=2)
+DENSE_FP4_DATASHEET_TFLOPS = 9000.0
+FP4_PER_BF16 = 4.0           # nominal dense FP4 : BF16 tensor ratio (9 : 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_traffic_from_profile():
+    """DRAM bytes per launch of the fprop GEMM from the committed ncu summary,
+    or None when the kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "gemm_nvf4_full.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"gemm_source_sha256:\s*([0-9a-f]{64})", text)
+    if not m or not h:
+        return None
+    src = open(os.path.join(ROOT, "nvfp4_bit_microscaled_b200", "csrc", "gemm.cu"), "rb").read()
+    if hashlib.sha256(src).hexdigest() != h.group(1):
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- our arm
+class Step:
+    """The hot path as individual C-ABI calls, with CUDA events around each
+    kernel group so per-kernel durations are measured inside the timed region."""
+
+    def __init__(self, X, W, dY, seed, record):
+        self.X, self.W, self.dY, self.seed = X, W, dY, seed
+        T, Cin = X.shape
+        Cout = W.shape[0]
+        dev = X.device
+        self.T, self.Cin, self.Cout = T, Cin, Cout
+        self.amax = torch.zeros(8, dtype=torch.float32, device=dev)
+        q = api.empty_qtensor
+        self.xr, self.wr, self.wc = q(T, Cin, dev), q(Cout, Cin, dev), q(Cin, Cout, dev)
+        self.xc, self.gr, self.gc = q(Cin, T, dev), q(T, Cout, dev), q(Cout, T, dev)
+        self.Y = torch.empty(T, Cout, dtype=torch.bfloat16, device=dev)
+        self.dX = torch.empty(T, Cin, dtype=torch.bfloat16, device=dev)
+        self.dW = torch.empty(Cout, Cin, dtype=torch.float32, device=dev)
+        self.record = record
+        self.events = []          # (kind, start, end)
+
+    def _ev(self, kind, fn):
+        if not self.record:
+            fn()
+            return
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        self.events.append((kind, s, e))
+
+    def __call__(self):
+        a = self.amax
+        X, W, dY = self.X, self.W, self.dY
+        # forward
+        self._ev("amax", lambda: api.amax(X, out=a[0:1]))
+        self._ev("quant_row", lambda: api.quantize(X, api.ROW, a[0:1], row_out=self.xr))
+        self._ev("amax", lambda: api.amax(W, out=a[1:2]))
+        self._ev("quant_2d", lambda: api.quantize(W, api.TWO_D, a[1:2], row_out=self.wr, col_out=self.wc))
+        self._ev("gemm_fprop", lambda: api.gemm(self.xr, self.wr, api.OUT_BF16, out=self.Y))
+        self._ev("amax_rht", lambda: api.amax(X, rht=True, out=a[2:3]))
+        self._ev("quant_col_rht", lambda: api.quantize(X, api.COL, a[2:3], rht=True, col_out=self.xc))
+        # backward
+        self._ev("amax", lambda: api.amax(dY, out=a[3:4]))
+        self._ev("quant_row_sr", lambda: api.quantize(dY, api.ROW, a[3:4], sr=True, seed=self.seed, row_out=self.gr))
+        self._ev("gemm_dgrad", lambda: api.gemm(self.gr, self.wc, api.OUT_BF16, out=self.dX))
+        self._ev("amax_rht", lambda: api.amax(dY, rht=True, out=a[4:5]))
+        self._ev("quant_col_rht_sr", lambda: api.quantize(dY, api.COL, a[4:5], rht=True, sr=True, seed=self.seed,
+                                                          col_out=self.gc))
+        self._ev("gemm_wgrad", lambda: api.gemm(self.gc, self.xc, api.OUT_F32, out=self.dW))
+
+    KERNELS_PER_STEP = 13  # 5 amax + 5 quantize + 3 GEMM kernels (no scale padding at these shapes)
+
+    def flops(self):
+        return 3 * 2.0 * self.T * self.Cin * self.Cout
+
+    def kernel_bytes(self):
+        """Algorithmic HBM bytes per kernel kind (reads + writes of the data the op must touch)."""
+        T, Ci, Co = self.T, self.Cin, self.Cout
+        q = lambda r, c: r * c / 2 + r * c / 16          # packed codes + one scale byte per 16
+        return {
+            "amax": 2.0 * (T * Ci + Ci * Co + T * Co),
+            "amax_rht": 2.0 * (T * Ci + T * Co),
+            "quant_row": 2.0 * T * Ci + q(T, Ci),
+            "quant_2d": 2.0 * Co * Ci + 2 * q(Co, Ci),
+            "quant_col_rht": 2.0 * T * Ci + q(T, Ci),
+            "quant_row_sr": 2.0 * T * Co + q(T, Co),
+            "quant_col_rht_sr": 2.0 * T * Co + q(T, Co),
+        }
+
+
+def gemm_flops(T, Ci, Co):
+    return {"gemm_fprop": 2.0 * T * Co * Ci, "gemm_dgrad": 2.0 * T * Ci * Co, "gemm_wgrad": 2.0 * Co * Ci * T}
+
+
+def run_ours(args, rank, world, device):
+    wl = WORKLOAD
+    T, Ci, Co = wl["T"], wl["Cin"], wl["Cout"]
+    seed = wl["seed"] + 1000 * rank      # every rank owns its own batch
+    X = synth.activations(T, Ci, seed, device=device)
+    W = synth.weights(Co, Ci, wl["seed"], device=device)
+    dY = synth.gradients(T, Co, seed, device=device)
+    torch.cuda.synchronize()
+    step = Step(X, W, dY, wl["sr_seed"], record=False)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    api.read_device_error(clear=True)
+
+    step.record = True
+    step.events = []
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                      else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[torch.cuda.current_device()]) as clk:
+        start.record()
+        for _ in range(args.steps):
+            step()
+        end.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = start.elapsed_time(end)
+    err = api.read_device_error(clear=True)
+    if err:
+        raise RuntimeError(f"device error word {err} after the timed region")
+
+    per_kind = {}
+    for kind, s, e in step.events:
+        per_kind.setdefault(kind, []).append(s.elapsed_time(e))
+    # each kind runs a fixed number of times per step; average per launch
+    avg_ms = {k: sum(v) / len(v) for k, v in per_kind.items()}
+    total_ms = {k: sum(v) / args.steps for k, v in per_kind.items()}
+
+    ms_max = ms_total
+    if world > 1:
+        t = torch.tensor([ms_total], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t[0])
+    ms_step = ms_max / args.steps
+    flops_step = step.flops()
+    value = flops_step * world / (ms_step * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    fp4_peak = FP4_PER_BF16 * peaks["bf16_tflops_sustained"]
+    gf = gemm_flops(T, Ci, Co)
+    g_ms = total_ms["gemm_fprop"] + total_ms["gemm_dgrad"] + total_ms["gemm_wgrad"]
+    gemm_tflops = {k: gf[k] / (avg_ms[k] * 1e-3) / 1e12 for k in gf}
+    fprop_achieved = gemm_tflops["gemm_fprop"]
+    kb = step.kernel_bytes()
+    q_kinds = ["quant_row", "quant_2d", "quant_col_rht", "quant_row_sr", "quant_col_rht_sr"]
+    q_bytes = sum(kb[k] for k in q_kinds)
+    q_ms = sum(total_ms[k] for k in q_kinds)
+    a_bytes = kb["amax"] + kb["amax_rht"]
+    a_ms = total_ms["amax"] + total_ms["amax_rht"]
+    hbm = peaks["hbm_gbs"]
+    traffic = gemm_traffic_from_profile()
+
+    kernels = {}
+    for k in avg_ms:
+        entry = {"ms_per_launch": round(avg_ms[k], 4), "launches_per_step": len(per_kind[k]) // args.steps}
+        if k in gf:
+            entry["tflops"] = round(gf[k] / (avg_ms[k] * 1e-3) / 1e12, 1)
+            entry["frac_fp4_peak"] = round(entry["tflops"] / fp4_peak, 4)
+        else:
+            nl = len(per_kind[k]) // args.steps
+            b = kb[k] / nl
+            entry["gbs"] = round(b / (avg_ms[k] * 1e-3) / 1e9, 1)
+            entry["frac_hbm"] = round(entry["gbs"] / hbm, 4)
+        kernels[k] = entry
+
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, fp32 accumulate)",
+        "data": "synthetic (seeded; X ~ N(0,1) with 0.1% outlier channels x100, W ~ N(0,0.02), "
+                "dY ~ N(0,1e-3) x per-row lognormal)",
+        "config": {
+            "workload": f"full linear fwd+bwd: T={T}, Cin={Ci}, Cout={Co} (FFN up-projection of a 12B hybrid "
+                        f"Mamba-Transformer); 3 GEMMs, 5 amax, 5 quantize kernels per step",
+            "T": T, "Cin": Ci, "Cout": Co,
+            "parallelism": f"independent batch per GPU x{world}",
+            "l2": "inputs larger than L2 (X 168 MB, W 210 MB, dY 671 MB; L2 126 MB): no flush needed",
+        },
+        "gemm": {
+            "tflops_gemm_only": round(sum(gf.values()) / (g_ms * 1e-3) / 1e12, 1),
+            "frac_fp4_peak": round(sum(gf.values()) / (g_ms * 1e-3) / 1e12 / fp4_peak, 4),
+            "frac_fp4_datasheet_9pf": round(sum(gf.values()) / (g_ms * 1e-3) / 1e12 / DENSE_FP4_DATASHEET_TFLOPS, 4),
+            "share_of_step": round(g_ms / ms_step, 3),
+        },
+        "quantize": {
+            "gbs": round(q_bytes / (q_ms * 1e-3) / 1e9, 1),
+            "frac_hbm": round(q_bytes / (q_ms * 1e-3) / 1e9 / hbm, 4),
+            "amax_gbs": round(a_bytes / (a_ms * 1e-3) / 1e9, 1),
+            "amax_frac_hbm": round(a_bytes / (a_ms * 1e-3) / 1e9 / hbm, 4),
+            "share_of_step": round((q_ms + a_ms) / ms_step, 3),
+        },
+        "kernels": kernels,
+        "roofline": {
+            "kernel": "gemm_nvf4_kernel (fprop, M=16384 N=20480 K=5120)",
+            "bound": "tensor",
+            "achieved": round(fprop_achieved, 1),
+            "peak": round(fp4_peak, 1),
+            "unit": "TFLOP/s",
+            "frac": round(fprop_achieved / fp4_peak, 4),
+            "peak_source": f"{peak_src}: 4 x bf16_tflops_sustained ({peaks['bf16_tflops_sustained']}) "
+                           f"(nominal dense FP4:BF16 = 9:2.25)",
+            "frac_of_datasheet_9pf": round(fprop_achieved / DENSE_FP4_DATASHEET_TFLOPS, 4),
+            "traffic": traffic,
+            "algorithmic_bytes": (T + Co) * Ci * 0.5625 + T * Co * 2,
+        },
+        "gpu_launches": Step.KERNELS_PER_STEP * args.steps,
+        "clocks": clk.summary(),
+    }
+    return result, (X, W, dY)
+
+
+def run_e2e(args, rank, world, device, tensors):
+    """Same metric through the public linear_fwd/linear_bwd calls with host
+    buffers: pinned host -> device copies of X, W, dY and device -> host copies
+    of Y, dX, dW inside the timed region."""
+    X, W, dY = tensors
+    T, Ci = X.shape
+    Co = W.shape[0]
+    hX, hW, hdY = (t.cpu().pin_memory() for t in (X, W, dY))
+    hY = torch.empty(T, Co, dtype=torch.bfloat16).pin_memory()
+    hdX = torch.empty(T, Ci, dtype=torch.bfloat16).pin_memory()
+    hdW = torch.empty(Co, Ci, dtype=torch.float32).pin_memory()
+    dXd, dWd, dYd = torch.empty_like(X), torch.empty_like(W), torch.empty_like(dY)
+    ws = api.LinearWorkspace(T, Ci, Co, device)
+    Y = torch.empty(T, Co, dtype=torch.bfloat16, device=device)
+    gX = torch.empty(T, Ci, dtype=torch.bfloat16, device=device)
+    gW = torch.empty(Co, Ci, dtype=torch.float32, device=device)
+
+    def one():
+        dXd.copy_(hX, non_blocking=True)
+        dWd.copy_(hW, non_blocking=True)
+        dYd.copy_(hdY, non_blocking=True)
+        api.linear_fwd(dXd, dWd, ws, Y=Y)
+        api.linear_bwd(dYd, ws, WORKLOAD["sr_seed"], dX=gX, dW=gW)
+        hY.copy_(Y, non_blocking=True)
+        hdX.copy_(gX, non_blocking=True)
+        hdW.copy_(gW, non_blocking=True)
+
+    steps = max(1, min(args.steps, 5))
+    for _ in range(min(args.warmup, 2)):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t[0])
+    ms_step = ms / steps
+    flops = 3 * 2.0 * T * Ci * Co
+    h2d = sum(t.numel() * t.element_size() for t in (hX, hW, hdY))
+    d2h = sum(t.numel() * t.element_size() for t in (hY, hdX, hdW))
+    return {"value": round(flops * world / (ms_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_step, 3),
+            "steps": steps}
+
+
+# --------------------------------------------------------------------------- reference arm
+def oracle_sample(seconds_target=15.0):
+    """The CPU oracle on a bounded sample of the same workload: the six
+    quantizations of a 64-token slice of the batch and W's first 256 rows, and
+    FP64 GEMM entries sampled from the three GEMMs.  Returns (TFLOP/s of GEMM
+    work, cores, description)."""
+    import numpy as np
+
+    import oracle as O
+
+    wl = WORKLOAD
+    Ci, Co = wl["Cin"], wl["Cout"]
+    Ts = 64
+    X = synth.activations(Ts, Ci, wl["seed"])
+    W = synth.weights(256, Ci, wl["seed"])
+    dY = synth.gradients(Ts, Co, wl["seed"])
+    rng = np.random.default_rng(0)
+    flops = 0.0
+    t0 = time.perf_counter()
+    ax, aw, ag = O.amax(X), O.amax(W), O.amax(dY)
+    axr, agr = O.amax_rht(X), O.amax_rht(dY)
+    cx, sx = O.quantize_row(X, ax)
+    cw, tw = O.quantize_2d(W, aw)
+    (cwr, swr), (cwc, swc) = O.expand_2d(cw, tw)
+    cxc, sxc = O.quantize_col(X, axr, rht=True)
+    cg, sg = O.quantize_row(dY, ag, sr=True, seed=wl["sr_seed"])
+    cgc, sgc = O.quantize_col(dY, agr, rht=True, sr=True, seed=wl["sr_seed"])
+    gs = lambda a: float(O.global_scales(a)[1])
+    n = 512
+    while True:
+        p1 = np.stack([rng.integers(0, Ts, n), rng.integers(0, 256, n)], 1)
+        O.gemm(cx, sx, gs(ax), cwr, swr, gs(aw), pairs=p1)                 # fprop entries, K = Cin
+        p3 = np.stack([rng.integers(0, Co, n), rng.integers(0, Ci, n)], 1)
+        O.gemm(cgc, sgc, gs(agr), cxc, sxc, gs(axr), pairs=p3)             # wgrad entries, K = Ts
+        flops += 2.0 * n * Ci + 2.0 * n * Ts
+        if time.perf_counter() - t0 > seconds_target:
+            break
+    dt = time.perf_counter() - t0
+    desc = (f"oracle (plain C, OpenMP) on host cores: amax/quantize of a {Ts}-token slice of X and dY and of "
+            f"W[:256], then FP64 GEMM entries sampled from fprop (K={Ci}) and wgrad (K={Ts}) for ~{seconds_target:.0f}s")
+    return flops / dt / 1e12, O.num_threads(), desc, dt
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    steps = []
+    per = max(3.0, 40.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(per)
+    for _ in range(args.steps):
+        v, cores, desc, dt = oracle_sample(per)
+        steps.append((v, dt))
+    value = statistics.mean(v for v, _ in steps)
+    ms = statistics.mean(dt for _, dt in steps) * 1e3
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 1),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64 GEMM on fp32-quantized operands",
+        "data": "synthetic (seeded)",
+        "config": {"workload": f"full linear fwd+bwd: T={WORKLOAD['T']}, Cin={WORKLOAD['Cin']}, "
+                               f"Cout={WORKLOAD['Cout']} (bounded sample, see cpu_baseline)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if world > 1:
+            import datetime
+            torch.distributed.init_process_group("gloo", timeout=datetime.timedelta(seconds=600))
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=device)
+    from nvfp4_bit_microscaled_b200 import build as libbuild
+    libbuild.build()
+
+    result, tensors = run_ours(args, rank, world, device)
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(args, rank, world, device, tensors)
+    del tensors
+    if rank == 0 and not args.no_cpu_baseline:
+        v, cores, desc, dt = oracle_sample(12.0)
+        result["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
