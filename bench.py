@@ -67,7 +67,7 @@ def gemm_traffic_from_profile():
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -75,6 +75,13 @@ class ClockSampler:
         self.gpu_index = gpu_index
         self.proc = None
         self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+        self.t0 = self.t1 = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def __enter__(self):
         try:
@@ -83,6 +90,7 @@ class ClockSampler:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
                  "-i", str(self.gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(1.0)          # let the sampler start before the timed region
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
@@ -99,19 +107,24 @@ class ClockSampler:
     def summary(self):
         if self.proc is None or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        import datetime
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    smax.append(float(parts[2]))
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    clk, clk_max = float(parts[2]), float(parts[3])
                 except ValueError:
                     continue
-                for n, v in zip(names, parts[5:9]):
+                if self.t0 is not None and not (self.t0 <= ts <= (self.t1 or ts)):
+                    continue
+                sm.append(clk)
+                smax.append(clk_max)
+                for n, v in zip(names, parts[6:10]):
                     if v.lower() == "active":
                         reasons.add(n)
         try:
@@ -122,6 +135,16 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def max_over_ranks(value, device, world):
+    """Max of a per-rank float over all ranks (device timing is reported as the
+    slowest rank's)."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t[0])
 
 
 # --------------------------------------------------------------------------- our arm
@@ -221,11 +244,13 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                       else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[torch.cuda.current_device()]) as clk:
+        clk.mark_start()
         start.record()
         for _ in range(args.steps):
             step()
         end.record()
         torch.cuda.synchronize()
+        clk.mark_end()
     if world > 1:
         torch.distributed.barrier()
     ms_total = start.elapsed_time(end)
@@ -240,11 +265,7 @@ def run_ours(args, rank, world, device):
     avg_ms = {k: sum(v) / len(v) for k, v in per_kind.items()}
     total_ms = {k: sum(v) / args.steps for k, v in per_kind.items()}
 
-    ms_max = ms_total
-    if world > 1:
-        t = torch.tensor([ms_total], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(t[0])
+    ms_max = max_over_ranks(ms_total, device, world)
     ms_step = ms_max / args.steps
     flops_step = step.flops()
     value = flops_step * world / (ms_step * 1e-3) / 1e12
@@ -370,11 +391,7 @@ def run_e2e(args, rank, world, device, tensors):
         one()
     e.record()
     torch.cuda.synchronize()
-    ms = s.elapsed_time(e)
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t[0])
+    ms = max_over_ranks(s.elapsed_time(e), device, world)
     ms_step = ms / steps
     flops = 3 * 2.0 * T * Ci * Co
     h2d = sum(t.numel() * t.element_size() for t in (hX, hW, hdY))
@@ -460,10 +477,71 @@ def run_reference(args, rank, world):
     }
 
 
+CASES = ("gemm", "amax", "amax_rht", "quant_row", "quant_row_sr", "quant_2d", "quant_col_rht",
+         "quant_col_rht_sr")
+
+
+def run_case(args):
+    """One kernel alone on a given shape (ncu captures, launch-shape sweeps).
+    gemm: --shape M,N,K (A activations, B weights, BF16 out); the others:
+    --shape R,C of the BF16 input.  Prints one JSON line."""
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    shape = [int(v) for v in args.shape.split(",")]
+    from nvfp4_bit_microscaled_b200 import build as libbuild
+    libbuild.build()
+    amax = torch.zeros(1, dtype=torch.float32, device=dev)
+    if args.case == "gemm":
+        M, N, K = shape
+        a_in, b_in = synth.activations(M, K, 5, device=dev), synth.weights(N, K, 5, device=dev)
+        qa, _ = api.quantize(a_in, api.ROW, api.amax(a_in))
+        qb, _ = api.quantize(b_in, api.ROW, api.amax(b_in))
+        D = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        fn = lambda: api.gemm(qa, qb, api.OUT_BF16, out=D)
+        work, unit = 2.0 * M * N * K, "TFLOP/s"
+    else:
+        R, C = shape
+        x = synth.gradients(R, C, 5, device=dev) if "sr" in args.case else synth.activations(R, C, 5, device=dev)
+        api.amax(x, rht="rht" in args.case, out=amax)
+        qbytes = R * C / 2 + R * C / 16
+        if args.case == "amax":
+            fn, work = (lambda: api.amax(x, out=amax)), 2.0 * R * C
+        elif args.case == "amax_rht":
+            fn, work = (lambda: api.amax(x, rht=True, out=amax)), 2.0 * R * C
+        elif args.case in ("quant_row", "quant_row_sr"):
+            q = api.empty_qtensor(R, C, dev)
+            sr = args.case.endswith("sr")
+            fn, work = (lambda: api.quantize(x, api.ROW, amax, sr=sr, seed=1, row_out=q)), 2.0 * R * C + qbytes
+        elif args.case == "quant_2d":
+            qr, qc = api.empty_qtensor(R, C, dev), api.empty_qtensor(C, R, dev)
+            fn, work = (lambda: api.quantize(x, api.TWO_D, amax, row_out=qr, col_out=qc)), 2.0 * R * C + 2 * qbytes
+        else:
+            q = api.empty_qtensor(C, R, dev)
+            sr = args.case.endswith("sr")
+            fn, work = (lambda: api.quantize(x, api.COL, amax, rht=True, sr=sr, seed=1, col_out=q)), \
+                2.0 * R * C + qbytes
+        unit = "GB/s"
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / args.steps
+    rate = work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
+    print(json.dumps({"case": args.case, "shape": shape, "ms_per_launch": round(ms, 4),
+                      "rate": round(rate, 1), "unit": unit}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--case", choices=CASES, help="time one kernel alone on --shape")
+    ap.add_argument("--shape", default="")
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
@@ -471,6 +549,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.case:
+        run_case(args)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
