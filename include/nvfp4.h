@@ -157,6 +157,33 @@ nvfp4_status nvfp4_linear_bwd(const void* dY, int64_t T, int64_t Cin, int64_t Co
                               float* dW, void* workspace, size_t workspace_bytes, nvfp4_stream_t stream);
 
 /*
+ * nvfp4_linear_fwd_noalloc -- nvfp4_linear_fwd for callers that cannot
+ * allocate device memory.  No counterpart on the pages: it is a property of
+ * this library, not of the method.
+ *
+ * Who needs it: code running while a stream is captured into a CUDA graph
+ * (allocation is not capturable), code in host callbacks or driver hooks where
+ * CUDA allocation calls are not allowed, and plugins whose host framework owns
+ * every device allocation.  Instead of a caller workspace it uses one scratch
+ * area of NVFP4_NOALLOC_SCRATCH_BYTES inside the library image (a __device__
+ * array that every GPU which loads the library holds until process exit).
+ *   - Computes exactly what nvfp4_linear_fwd computes (same kernels, same
+ *     order); Y is written as there.  X, W, Y as in nvfp4_linear_fwd.
+ *   - Returns NVFP4_ERR_WORKSPACE, before enqueuing anything, when
+ *     nvfp4_linear_workspace_bytes(T, Cin, Cout) exceeds the scratch size.
+ *   - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
+ *   - Its first call on a device looks up the scratch address on that device
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call shares the one scratch area and leaves its contents behind
+ *     (the quantized operands of the last call); each call rewrites what it
+ *     reads.  Calls whose GPU work overlaps (other streams, other threads on
+ *     the same device) race on the scratch: serialize them.
+ */
+#define NVFP4_NOALLOC_SCRATCH_BYTES (16u << 20)
+nvfp4_status nvfp4_linear_fwd_noalloc(const void* X, const void* W, int64_t T, int64_t Cin, int64_t Cout, void* Y,
+                                      nvfp4_stream_t stream);
+
+/*
  * The quantized operands inside a linear workspace (descriptors only; the
  * memory is the workspace's).  which: 0 X row, 1 W row, 2 W column, 3 X column
  * (RHT), 4 dY row (SR), 5 dY column (RHT + SR).

@@ -44,6 +44,7 @@ PROTOTYPES = {
     "nvfp4_linear_fwd": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _c.c_size_t, _vp]),
     "nvfp4_linear_bwd": (_int, [_vp, _i64, _i64, _i64, _u64, _vp, _vp, _vp, _c.c_size_t, _vp]),
     "nvfp4_linear_workspace_tensor": (_int, [_vp, _i64, _i64, _i64, _int, _tp]),
+    "nvfp4_linear_fwd_noalloc": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp]),
     "nvfp4_read_device_error": (_int, [_c.POINTER(_c.c_uint), _int]),
     "nvfp4_wait_probe": (_int, [_u32, _vp]),
     "nvfp4_rht_sign_mask": (_u32, []),

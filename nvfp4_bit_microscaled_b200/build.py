@@ -12,7 +12,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnvfp4.so")
-SOURCES = ["amax.cu", "quantize.cu", "gemm.cu", "api.cu"]
+SOURCES = ["amax.cu", "quantize.cu", "gemm.cu", "api.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 PUBLIC_HEADER = os.path.join(os.path.dirname(HERE), "include", "nvfp4.h")
 
