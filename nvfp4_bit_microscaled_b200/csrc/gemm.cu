@@ -10,16 +10,21 @@
 // (Y = X W^T), dgrad (dX = dY W) and wgrad (dW = dY^T X): every operand is
 // stored K-major (the contracted dimension contiguous).
 //
-// Design (persistent, warp-specialised, one CTA per SM):
-//   warp 0  TMA producer: A tile 128 x 256 and B tile 256 x 256 (packed FP4,
-//           128-byte swizzle) plus their 128x4 scale tiles (1-D bulk copies)
-//           into a 4-stage shared-memory ring guarded by mbarriers;
-//   warp 1  MMA issuer: copies the stage's scales to tensor memory
-//           (tcgen05.cp) and issues four tcgen05.mma kind::mxf4nvf4 (K = 64
-//           each, 16-element E4M3 block scales) into a 128 x 256 FP32
-//           accumulator in tensor memory; tcgen05.commit frees the stage;
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator, x alpha, store FP32
-//           or BF16; then hand the accumulator back to the MMA issuer.
+// Design (persistent, warp-specialised, one CTA per SM, 14 warps):
+//   warp 0      TMA producer: A tile 128 x 256 and B tile 256 x 256 (packed
+//               FP4, 128-byte swizzle) plus their 128x4 scale tiles (1-D bulk
+//               copies) into a 4-stage shared-memory ring guarded by mbarriers;
+//   warps 10-13 scale warps: for each stage, read the scale tiles from shared
+//               memory and write them into that stage's tensor-memory scale
+//               buffer (tcgen05.st, one warp per 32-lane quarter), so the
+//               tensor pipe never spends time copying scales;
+//   warp 1      MMA issuer: four tcgen05.mma kind::mxf4nvf4 per stage (K = 64
+//               each, 16-element UE4M3 block scales from tensor memory) into a
+//               128 x 256 FP32 accumulator in tensor memory; tcgen05.commit
+//               frees the stage and, after the last stage, the accumulator;
+//   warps 2-9   epilogue, two warps per 32-lane quarter (128 columns each):
+//               tcgen05.ld of the accumulator, x alpha, hand the accumulator
+//               back, then store FP32 or BF16.
 // Every mbarrier wait is bounded; on a timeout the kernel records an error
 // word, lets in-flight copies and MMAs land, frees tensor memory and returns.
 #include <cuda.h>
@@ -49,9 +54,14 @@ constexpr uint32_t OFF_SFA = OFF_B + STAGES * B_BYTES;
 constexpr uint32_t OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
 constexpr uint32_t OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;        // + barriers + alignment slack
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 448;
+constexpr int EPI_WARP0 = 2, NUM_EPI_WARPS = 8, SF_WARP0 = 10, NUM_SF_WARPS = 4;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 256 + 16;
+// Tensor memory: accumulator in columns [0, 256); one scale buffer per stage
+// (48 columns: 16 for A, 32 for B).  A stage's buffer is rewritten only after
+// the stage's shared memory was refilled, i.e. after the MMAs that read the
+// previous scales completed.
+constexpr uint32_t ACC_COL = 0, SF_COL = 256, SF_BUF_COLS = 48, SFB_OFF = 16;
 constexpr int GROUP_M = 16;                                  // tile raster: 16 M-tiles share B tiles in L2
 
 // Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1), K-major,
@@ -84,7 +94,8 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* mma_done = acc_empty + 1;
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(mma_done + 1);
+  uint64_t* sf_full = mma_done + 1;           // [STAGES]: scale warps -> MMA issuer
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sf_full + STAGES);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -99,8 +110,9 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
+    mbar_init(acc_empty, NUM_EPI_WARPS);
     mbar_init(mma_done, 1);
+    for (int s = 0; s < STAGES; ++s) mbar_init(&sf_full[s], NUM_SF_WARPS);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tmA);
@@ -152,7 +164,6 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     int stage = 0;
     uint32_t phase = 0, acc_phase = 0;
     const uint32_t a_base = smem_u32(smem + OFF_A), b_base = smem_u32(smem + OFF_B);
-    const uint32_t sfa_base = smem_u32(smem + OFF_SFA), sfb_base = smem_u32(smem + OFF_SFB);
     for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
       const TileCoord tc = tile_coord(t, num_m, num_n);
       const bool second_half = tc.n * BN + 128 < N;
@@ -161,23 +172,19 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       tc_fence_after();
       bool ok = true;
       for (int kt = 0; kt < num_kt; ++kt) {
-        if (!mbar_wait(&full[stage], phase, kErrWaitFull)) { ok = false; break; }
+        if (!mbar_wait(&full[stage], phase, kErrWaitFull) || !mbar_wait(&sf_full[stage], phase, kErrWaitFull)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const int nkb = min(KB_PER_STAGE, katoms - kt * KB_PER_STAGE);
-        const uint32_t sfa_s = sfa_base + stage * SFA_BYTES, sfb_s = sfb_base + stage * SFB_BYTES;
-        for (int kb = 0; kb < nkb; ++kb) {
-          tmem_cp_32x128b_x4(tmem + SFA_COL + 4 * kb, smem_desc(sfa_s + 512 * kb, 16, 128, 0));
-          tmem_cp_32x128b_x4(tmem + SFB_COL + 8 * kb, smem_desc(sfb_s + 512 * kb, 16, 128, 0));
-          if (second_half)
-            tmem_cp_32x128b_x4(tmem + SFB_COL + 8 * kb + 4,
-                               smem_desc(sfb_s + KB_PER_STAGE * 512 + 512 * kb, 16, 128, 0));
-        }
+        const uint32_t sfa_t = tmem + SF_COL + stage * SF_BUF_COLS, sfb_t = sfa_t + SFB_OFF;
         const uint64_t adesc = smem_desc(a_base + stage * A_BYTES, 16, 1024, 2);
         const uint64_t bdesc = smem_desc(b_base + stage * B_BYTES, 16, 1024, 2);
         for (int kb = 0; kb < nkb; ++kb) {
           // +32 bytes along K inside the 128-byte swizzle row = +2 in the 16-byte address field
-          mma_nvf4(tmem + ACC_COL, adesc + 2 * kb, bdesc + 2 * kb, idesc, tmem + SFA_COL + 4 * kb,
-                   tmem + SFB_COL + 8 * kb, (kt | kb) != 0);
+          mma_nvf4(tmem + ACC_COL, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa_t + 4 * kb, sfb_t + 8 * kb,
+                   (kt | kb) != 0);
         }
         tc_commit(&empty[stage]);
         if (++stage == STAGES) stage = 0, phase ^= 1u;
@@ -189,57 +196,111 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     // Let every MMA this thread issued finish before tensor memory is freed.
     tc_commit(mma_done);
     mbar_wait(mma_done, 0, kErrWaitAccFull);
-  } else if (warp >= 2) {
+  } else if (warp >= SF_WARP0) {
+    // ------------------------------------------------------------ scale warps
+    // Tensor-memory layout the block-scaled MMA reads (M or N = 128 per 128x4
+    // tile): lane l, column 4*kb + c holds the four scales of row 32*c + l%32
+    // for K-step kb, replicated over the four 32-lane quarters.  Row l%32 of a
+    // 512-byte tile is exactly those 16 bytes, so each lane loads one 16-byte
+    // row per tile and each warp writes its own lane quarter.
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+      const TileCoord tc = tile_coord(t, num_m, num_n);
+      const bool second_half = tc.n * BN + 128 < N;
+      bool ok = true;
+      for (int kt = 0; kt < num_kt; ++kt) {
+        if (!mbar_wait(&full[stage], phase, kErrWaitFull)) { ok = false; break; }
+        const int nkb = min(KB_PER_STAGE, katoms - kt * KB_PER_STAGE);
+        const uint8_t* sa = smem + OFF_SFA + stage * SFA_BYTES + lane * 16;
+        const uint8_t* sb = smem + OFF_SFB + stage * SFB_BYTES + lane * 16;
+        uint32_t ra[16], rb[32];
+#pragma unroll
+        for (int kb = 0; kb < KB_PER_STAGE; ++kb) {
+          const uint4 va = kb < nkb ? *reinterpret_cast<const uint4*>(sa + 512 * kb) : make_uint4(0, 0, 0, 0);
+          const uint4 v0 = kb < nkb ? *reinterpret_cast<const uint4*>(sb + 512 * kb) : make_uint4(0, 0, 0, 0);
+          const uint4 v1 = (kb < nkb && second_half)
+                               ? *reinterpret_cast<const uint4*>(sb + KB_PER_STAGE * 512 + 512 * kb)
+                               : make_uint4(0, 0, 0, 0);
+          ra[4 * kb + 0] = va.x; ra[4 * kb + 1] = va.y; ra[4 * kb + 2] = va.z; ra[4 * kb + 3] = va.w;
+          rb[8 * kb + 0] = v0.x; rb[8 * kb + 1] = v0.y; rb[8 * kb + 2] = v0.z; rb[8 * kb + 3] = v0.w;
+          rb[8 * kb + 4] = v1.x; rb[8 * kb + 5] = v1.y; rb[8 * kb + 6] = v1.z; rb[8 * kb + 7] = v1.w;
+        }
+        const uint32_t sfa_t = tmem + lane_base + SF_COL + stage * SF_BUF_COLS;
+        tmem_st_32x32b_x16(sfa_t, ra);
+        tmem_st_32x32b_x32(sfa_t + SFB_OFF, rb);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_full[stage]);
+        if (++stage == STAGES) stage = 0, phase ^= 1u;
+      }
+      if (!ok) { *abort_flag = 1; break; }
+    }
+  } else if (warp >= EPI_WARP0) {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;  // tensor-memory lanes this warp may read
+    const int quarter = warp & 3;                   // tensor-memory lanes this warp may read
+    const int col_half = (warp - EPI_WARP0) >> 2;   // columns [128 * col_half, +128) of the tile
     const float alpha = __fmul_rn(__ldg(gsa), __ldg(gsb));
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
       const TileCoord tc = tile_coord(t, num_m, num_n);
       if (!mbar_wait(acc_full, acc_phase, kErrWaitAccFull)) { *abort_flag = 1; break; }
       tc_fence_after();
       const int row = tc.m * BM + quarter * 32 + lane;
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        const int col0 = tc.n * BN + ch * 32;
-        if (col0 >= N) break;
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ACC_COL + ch * 32, r);
-        tmem_ld_wait();
-        if (row < M) {
-          const int ncols = min(32, N - col0);
-          if (out_bf16) {
-            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(D) + static_cast<int64_t>(row) * ldd + col0;
+      const int col_base = tc.n * BN + col_half * 128;
+      if (out_bf16) {
+        // read all 128 columns (packed to BF16 pairs), release the accumulator, then store
+        uint32_t packed[64];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (v * 8 < ncols) {
-                uint32_t p[4];
+        for (int ch = 0; ch < 4; ++ch) {
+          if (col_base + ch * 32 < N) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(tmem + lane_base + ACC_COL + col_half * 128 + ch * 32, r);
+            tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[v * 8 + 2 * e]), alpha),
-                                                           __fmul_rn(__uint_as_float(r[v * 8 + 2 * e + 1]), alpha));
-                  p[e] = *reinterpret_cast<uint32_t*>(&h);
-                }
-                reinterpret_cast<uint4*>(dst)[v] = make_uint4(p[0], p[1], p[2], p[3]);
-              }
-            }
-          } else {
-            float* dst = static_cast<float*>(D) + static_cast<int64_t>(row) * ldd + col0;
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              if (v * 4 < ncols) {
-                reinterpret_cast<float4*>(dst)[v] =
-                    make_float4(__fmul_rn(__uint_as_float(r[4 * v + 0]), alpha),
-                                __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
-                                __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha),
-                                __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
-              }
+            for (int e = 0; e < 16; ++e) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
+                                                       __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
+              packed[16 * ch + e] = *reinterpret_cast<uint32_t*>(&h);
             }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+        if (row < M) {
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(D) + static_cast<int64_t>(row) * ldd + col_base;
+#pragma unroll
+          for (int v = 0; v < 16; ++v)
+            if (col_base + v * 8 < N)
+              reinterpret_cast<uint4*>(dst)[v] =
+                  make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+        }
+      } else {
+        for (int ch = 0; ch < 4; ++ch) {
+          const int col0 = col_base + ch * 32;
+          if (col0 >= N) break;
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + ACC_COL + col_half * 128 + ch * 32, r);
+          tmem_ld_wait();
+          if (row < M) {
+            float* dst = static_cast<float*>(D) + static_cast<int64_t>(row) * ldd + col0;
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              if (col0 + v * 4 < N)
+                reinterpret_cast<float4*>(dst)[v] = make_float4(__fmul_rn(__uint_as_float(r[4 * v + 0]), alpha),
+                                                                __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
+                                                                __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha),
+                                                                __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
       acc_phase ^= 1u;
     }
   }

@@ -57,12 +57,12 @@ __device__ __forceinline__ void fwht16(float (&v)[16]) {
 // Scale bytes of lanes 4j..4j+3 form one 32-bit word of the 128x4 tile layout.
 // ---------------------------------------------------------------------------
 template <bool SR>
-__global__ void __launch_bounds__(256) quant_row_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+__global__ void __launch_bounds__(256, SR ? 3 : 4) quant_row_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
                                                           int64_t ld, const float* __restrict__ amax_dev,
                                                           uint32_t k0, uint32_t k1, uint8_t* __restrict__ data,
                                                           uint8_t* __restrict__ sf, int64_t sp,
                                                           float* __restrict__ gs_out) {
-  constexpr int U = 2;  // items in flight per warp
+  constexpr int U = SR ? 1 : 2;  // items in flight per warp
   const float amax = __ldg(amax_dev);
   const float s_enc = encode_scale(amax);
   if (blockIdx.x == 0 && threadIdx.x == 0 && gs_out) *gs_out = decode_scale(amax);
@@ -129,16 +129,18 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const uint16_t* __restri
 // output.  Thread item: 64 tokens x 4 channels.  Each 16-token block of a
 // channel is optionally rotated by Q = 1/4 H16 diag(s) before it is scaled.
 // Loads: 16 rows x 8 bytes per block (coalesced along the row across the
-// warp); stores: 32 bytes of codes and one 4-byte scale word per channel.
+// warp); stores: 8 bytes of codes per channel and block as each block is done
+// (the four blocks of a 64-token item fill one 32-byte sector), one 4-byte
+// scale word per channel per item.
 // SR word for element (t, c): Philox counter (t*C + c) >> 2, so one call
 // serves the four channels of a row.
 // ---------------------------------------------------------------------------
 template <bool RHT, bool SR>
-__global__ void __launch_bounds__(256) quant_col_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
-                                                          int64_t ld, const float* __restrict__ amax_dev,
-                                                          uint32_t sign_mask, uint32_t k0, uint32_t k1,
-                                                          uint8_t* __restrict__ data, uint8_t* __restrict__ sf,
-                                                          int64_t sp, float* __restrict__ gs_out) {
+__global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+                                                             int64_t ld, const float* __restrict__ amax_dev,
+                                                             uint32_t sign_mask, uint32_t k0, uint32_t k1,
+                                                             uint8_t* __restrict__ data, uint8_t* __restrict__ sf,
+                                                             int64_t sp, float* __restrict__ gs_out) {
   const float amax = __ldg(amax_dev);
   const float s_enc = encode_scale(amax);
   if (blockIdx.x == 0 && threadIdx.x == 0 && gs_out) *gs_out = decode_scale(amax);
@@ -147,20 +149,14 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const uint16_t* __restri
   const int64_t ng = C >> 2;
   const int64_t items = nq * ng;
   const int64_t half_r = R >> 1;
-  const bool vec_store = (R & 31) == 0;
 
   for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items;
        it += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t q = it / ng, g = it - q * ng;
     const int64_t c0 = g * 4, t0 = q * 64;
     const int nb = static_cast<int>((S - 4 * q) < 4 ? (S - 4 * q) : 4);
-    uint32_t lo[4][4], hi[4][4];  // [channel][block] codes (8 nibbles each half)
     uint32_t sfw[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-    for (int tb = 0; tb < 4; ++tb) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) lo[c][tb] = hi[c][tb] = 0u;
-      if (tb >= nb) continue;
+    for (int tb = 0; tb < nb; ++tb) {
       const int64_t tbase = t0 + 16 * tb;
       float v[4][16];
 #pragma unroll
@@ -188,6 +184,7 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const uint16_t* __restri
         r[c] = bs.r;
         sfw[c] |= bs.sf << (8 * tb);
       }
+      uint32_t lo[4] = {0u, 0u, 0u, 0u}, hi[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int i = 0; i < 16; i += 2) {
         float y0[4], y1[4];
@@ -208,28 +205,16 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const uint16_t* __restri
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const uint32_t byte = f32x2_to_e2m1x2(y0[c], y1[c]) << sh;
-          if (i < 8) lo[c][tb] |= byte; else hi[c][tb] |= byte;
+          if (i < 8) lo[c] |= byte; else hi[c] |= byte;
         }
       }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        lo[c][tb] = clear_negative_zero(lo[c][tb]);
-        hi[c][tb] = clear_negative_zero(hi[c][tb]);
-      }
+      for (int c = 0; c < 4; ++c)
+        reinterpret_cast<uint2*>(data + (c0 + c) * half_r + t0 / 2)[tb] =
+            make_uint2(clear_negative_zero(lo[c]), clear_negative_zero(hi[c]));
     }
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint8_t* dst = data + (c0 + c) * half_r + t0 / 2;
-      if (nb == 4 && vec_store) {
-        reinterpret_cast<uint4*>(dst)[0] = make_uint4(lo[c][0], hi[c][0], lo[c][1], hi[c][1]);
-        reinterpret_cast<uint4*>(dst)[1] = make_uint4(lo[c][2], hi[c][2], lo[c][3], hi[c][3]);
-      } else {
-#pragma unroll
-        for (int tb = 0; tb < 4; ++tb)
-          if (tb < nb) reinterpret_cast<uint2*>(dst)[tb] = make_uint2(lo[c][tb], hi[c][tb]);
-      }
-      *reinterpret_cast<uint32_t*>(sf + sf_offset(c0 + c, 4 * q, sp)) = sfw[c];
-    }
+    for (int c = 0; c < 4; ++c) *reinterpret_cast<uint32_t*>(sf + sf_offset(c0 + c, 4 * q, sp)) = sfw[c];
   }
 }
 
