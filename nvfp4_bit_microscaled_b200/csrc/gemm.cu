@@ -172,7 +172,9 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       tc_fence_after();
       bool ok = true;
       for (int kt = 0; kt < num_kt; ++kt) {
-        if (!mbar_wait(&full[stage], phase, kErrWaitFull) || !mbar_wait(&sf_full[stage], phase, kErrWaitFull)) {
+        // the scale warps arrive only after the stage's data landed, so one
+        // wait covers both the operands and the scales
+        if (!mbar_wait(&sf_full[stage], phase, kErrWaitFull)) {
           ok = false;
           break;
         }
@@ -310,6 +312,262 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
+// ===========================================================================
+// CTA-pair kernel (cta_group::2) for M and N multiples of 256.
+//
+// A cluster of two CTAs computes a 256 x 256 tile with one pair MMA per K-step
+// (M = 256 over both CTAs' tensor memory).  Each CTA loads its own 128 rows of
+// A and its own 128 rows of B, so per SM a stage moves 38 KiB for the same MMA
+// work that costs 54 KiB in the single-CTA kernel; the rest of the design is
+// the single-CTA kernel's (scale warps, 8 epilogue warps).  Every CTA writes
+// the scales of all 256 B rows into its own tensor memory, as the pair MMA
+// reads B's scales from each CTA.  The leader (cluster rank 0) issues the
+// MMAs; both CTAs' loads, scale writes and epilogues report to the leader's
+// barriers, and the leader's commits arrive in both CTAs.
+// ===========================================================================
+constexpr int P_STAGES = 5;
+constexpr uint32_t P_A_BYTES = 128 * BK_BYTES;                 // 16 KiB (own A rows)
+constexpr uint32_t P_B_BYTES = 128 * BK_BYTES;                 // 16 KiB (own half of B)
+constexpr uint32_t P_SFA_BYTES = KB_PER_STAGE * 512;           // 2 KiB
+constexpr uint32_t P_SFB_BYTES = 2 * KB_PER_STAGE * 512;       // 4 KiB (both halves of B)
+constexpr uint32_t P_OFF_A = 0;
+constexpr uint32_t P_OFF_B = P_OFF_A + P_STAGES * P_A_BYTES;
+constexpr uint32_t P_OFF_SFA = P_OFF_B + P_STAGES * P_B_BYTES;
+constexpr uint32_t P_OFF_SFB = P_OFF_SFA + P_STAGES * P_SFA_BYTES;
+constexpr uint32_t P_OFF_BAR = P_OFF_SFB + P_STAGES * P_SFB_BYTES;
+constexpr uint32_t P_SMEM_BYTES = P_OFF_BAR + 512 + 1024;
+constexpr int P_GROUP_M = 8;
+
+// kind::mxf4nvf4, A/B E2M1 K-major, UE4M3 scales, M = 256 (pair), N = 256.
+__host__ __device__ constexpr uint32_t make_idesc_pair() {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(256 >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
+                      const float* __restrict__ gsa, const float* __restrict__ gsb, int M, int N, int K,
+                      void* __restrict__ D, int out_bf16, int64_t ldd) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_OFF_BAR);   // leader: A/B bytes of both CTAs
+  uint64_t* empty = full + P_STAGES;                                 // both: leader's commit
+  uint64_t* sfd_full = empty + P_STAGES;                             // both: own scale bytes landed
+  uint64_t* sf_full = sfd_full + P_STAGES;                           // leader: 8 scale warps done
+  uint64_t* acc_full = sf_full + P_STAGES;                           // both: leader's commit
+  uint64_t* acc_empty = acc_full + 1;                                // leader: 16 epilogue warps
+  uint64_t* mma_done = acc_empty + 1;                                // leader
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(mma_done + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+  const int num_m = M / 256, num_n = N / 256;
+  const int num_tiles = num_m * num_n;
+  const int katoms = (K + 63) / 64;
+  const int num_kt = (K + 255) / 256;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sfd_full[s], 1);
+      mbar_init(&sf_full[s], 2 * NUM_SF_WARPS);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * NUM_EPI_WARPS);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) tmem_alloc_pair(const_cast<uint32_t*>(tmem_slot), TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // leader-CTA cluster addresses of the barriers the peer reports to
+  const uint32_t full_l = mapa_shared(smem_u32(full), 0), sf_full_l = mapa_shared(smem_u32(sf_full), 0);
+  const uint32_t acc_empty_l = mapa_shared(smem_u32(acc_empty), 0);
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_parity[P_STAGES];
+    bool issued[P_STAGES];
+    for (int s = 0; s < P_STAGES; ++s) issued[s] = false, issued_parity[s] = 0;
+    for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
+      const int per_group = P_GROUP_M * num_n, grp = t / per_group, first_m = grp * P_GROUP_M;
+      const int gsize = min(num_m - first_m, P_GROUP_M), within = t - grp * per_group;
+      const int tm = first_m + within % gsize, tn = within / gsize;
+      for (int kt = 0; kt < num_kt; ++kt) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, kErrWaitEmpty)) { *abort_flag = 1; break; }
+        const int nkb = min(KB_PER_STAGE, katoms - kt * KB_PER_STAGE);
+        const uint32_t sf_bytes = static_cast<uint32_t>(nkb) * 512u;
+        if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (P_A_BYTES + P_B_BYTES));
+        tma_load_2d_pair(smem + P_OFF_A + stage * P_A_BYTES, &tmA, full_l + stage * 8, kt * BK_BYTES,
+                         tm * 256 + 128 * static_cast<int>(rank));
+        tma_load_2d_pair(smem + P_OFF_B + stage * P_B_BYTES, &tmB, full_l + stage * 8, kt * BK_BYTES,
+                         tn * 256 + 128 * static_cast<int>(rank));
+        mbar_arrive_expect_tx(&sfd_full[stage], 3 * sf_bytes);
+        bulk_load(smem + P_OFF_SFA + stage * P_SFA_BYTES,
+                  sfa + (static_cast<int64_t>(2 * tm + rank) * katoms + kt * KB_PER_STAGE) * 512, sf_bytes,
+                  &sfd_full[stage]);
+        for (int h = 0; h < 2; ++h)
+          bulk_load(smem + P_OFF_SFB + stage * P_SFB_BYTES + h * KB_PER_STAGE * 512,
+                    sfb + (static_cast<int64_t>(2 * tn + h) * katoms + kt * KB_PER_STAGE) * 512, sf_bytes,
+                    &sfd_full[stage]);
+        issued[stage] = true;
+        issued_parity[stage] = phase;
+        if (++stage == P_STAGES) stage = 0, phase ^= 1u;
+      }
+    }
+    // Let every copy this thread started land before the CTA can exit.
+    for (int s = 0; s < P_STAGES; ++s)
+      if (issued[s]) mbar_wait(&sfd_full[s], issued_parity[s], kErrWaitFull);
+    if (rank == 0)
+      for (int s = 0; s < P_STAGES; ++s)
+        if (issued[s]) mbar_wait_cluster(&full[s], issued_parity[s], kErrWaitFull);
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    int stage = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    const uint32_t a_base = smem_u32(smem + P_OFF_A), b_base = smem_u32(smem + P_OFF_B);
+    const uint32_t idesc = make_idesc_pair();
+    for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
+      if (!mbar_wait_cluster(acc_empty, acc_phase ^ 1u, kErrWaitAccEmpty)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      bool ok = true;
+      for (int kt = 0; kt < num_kt; ++kt) {
+        // the leader's scale warps arrive only after both CTAs' operands
+        // landed (full), so one wait covers operands and scales
+        if (!mbar_wait_cluster(&sf_full[stage], phase, kErrWaitFull)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int nkb = min(KB_PER_STAGE, katoms - kt * KB_PER_STAGE);
+        const uint32_t sfa_t = tmem + SF_COL + stage * SF_BUF_COLS, sfb_t = sfa_t + SFB_OFF;
+        const uint64_t adesc = smem_desc(a_base + stage * P_A_BYTES, 16, 1024, 2);
+        const uint64_t bdesc = smem_desc(b_base + stage * P_B_BYTES, 16, 1024, 2);
+        for (int kb = 0; kb < nkb; ++kb)
+          mma_nvf4_pair(tmem + ACC_COL, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa_t + 4 * kb, sfb_t + 8 * kb,
+                        (kt | kb) != 0);
+        tc_commit_pair_mc(&empty[stage], 0x3);
+        if (++stage == P_STAGES) stage = 0, phase ^= 1u;
+      }
+      if (!ok) { *abort_flag = 1; break; }
+      tc_commit_pair_mc(acc_full, 0x3);
+      acc_phase ^= 1u;
+    }
+    tc_commit_pair(mma_done);
+    mbar_wait(mma_done, 0, kErrWaitAccFull);
+  } else if (warp >= SF_WARP0) {
+    // ------------------------------------------------------------ scale warps (both CTAs)
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
+      bool ok = true;
+      for (int kt = 0; kt < num_kt; ++kt) {
+        if (!mbar_wait(&sfd_full[stage], phase, kErrWaitFull) ||
+            (rank == 0 && !mbar_wait_cluster(&full[stage], phase, kErrWaitFull))) {
+          ok = false;
+          break;
+        }
+        const int nkb = min(KB_PER_STAGE, katoms - kt * KB_PER_STAGE);
+        const uint8_t* sa = smem + P_OFF_SFA + stage * P_SFA_BYTES + lane * 16;
+        const uint8_t* sb = smem + P_OFF_SFB + stage * P_SFB_BYTES + lane * 16;
+        uint32_t ra[16], rb[32];
+#pragma unroll
+        for (int kb = 0; kb < KB_PER_STAGE; ++kb) {
+          const uint4 va = kb < nkb ? *reinterpret_cast<const uint4*>(sa + 512 * kb) : make_uint4(0, 0, 0, 0);
+          const uint4 v0 = kb < nkb ? *reinterpret_cast<const uint4*>(sb + 512 * kb) : make_uint4(0, 0, 0, 0);
+          const uint4 v1 =
+              kb < nkb ? *reinterpret_cast<const uint4*>(sb + KB_PER_STAGE * 512 + 512 * kb) : make_uint4(0, 0, 0, 0);
+          ra[4 * kb + 0] = va.x; ra[4 * kb + 1] = va.y; ra[4 * kb + 2] = va.z; ra[4 * kb + 3] = va.w;
+          rb[8 * kb + 0] = v0.x; rb[8 * kb + 1] = v0.y; rb[8 * kb + 2] = v0.z; rb[8 * kb + 3] = v0.w;
+          rb[8 * kb + 4] = v1.x; rb[8 * kb + 5] = v1.y; rb[8 * kb + 6] = v1.z; rb[8 * kb + 7] = v1.w;
+        }
+        const uint32_t sfa_t = tmem + lane_base + SF_COL + stage * SF_BUF_COLS;
+        tmem_st_32x32b_x16(sfa_t, ra);
+        tmem_st_32x32b_x32(sfa_t + SFB_OFF, rb);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(sf_full_l + stage * 8);
+        if (++stage == P_STAGES) stage = 0, phase ^= 1u;
+      }
+      if (!ok) { *abort_flag = 1; break; }
+    }
+  } else if (warp >= EPI_WARP0) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;
+    const int col_half = (warp - EPI_WARP0) >> 2;
+    const float alpha = __fmul_rn(__ldg(gsa), __ldg(gsb));
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
+      const int per_group = P_GROUP_M * num_n, grp = t / per_group, first_m = grp * P_GROUP_M;
+      const int gsize = min(num_m - first_m, P_GROUP_M), within = t - grp * per_group;
+      const int tm = first_m + within % gsize, tn = within / gsize;
+      if (!mbar_wait_cluster(acc_full, acc_phase, kErrWaitAccFull)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      const int row = tm * 256 + 128 * static_cast<int>(rank) + quarter * 32 + lane;
+      const int col_base = tn * 256 + col_half * 128;
+      if (out_bf16) {
+        uint32_t packed[64];
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + ACC_COL + col_half * 128 + ch * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
+                                                     __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
+            packed[16 * ch + e] = *reinterpret_cast<uint32_t*>(&h);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty_l);
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(D) + static_cast<int64_t>(row) * ldd + col_base;
+#pragma unroll
+        for (int v = 0; v < 16; ++v)
+          reinterpret_cast<uint4*>(dst)[v] =
+              make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+      } else {
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + ACC_COL + col_half * 128 + ch * 32, r);
+          tmem_ld_wait();
+          float* dst = static_cast<float*>(D) + static_cast<int64_t>(row) * ldd + col_base + ch * 32;
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            reinterpret_cast<float4*>(dst)[v] = make_float4(__fmul_rn(__uint_as_float(r[4 * v + 0]), alpha),
+                                                            __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
+                                                            __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha),
+                                                            __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty_l);
+      }
+      acc_phase ^= 1u;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its peer may still signal its barriers
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, TMEM_COLS);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -343,9 +601,51 @@ bool make_operand_map(CUtensorMap* tm, const void* data, int64_t rows, int64_t K
 cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a_gs, const void* b_data,
                         const void* b_scales, const float* b_gs, int64_t M, int64_t N, int64_t K, void* D,
                         int out_bf16, int64_t ldd, int num_sms, cudaStream_t s) {
+  const bool pair = (M % 256 == 0) && (N % 256 == 0);
   CUtensorMap tmA, tmB;
-  if (!make_operand_map(&tmA, a_data, M, K, BM) || !make_operand_map(&tmB, b_data, N, K, BN))
+  if (!make_operand_map(&tmA, a_data, M, K, BM) || !make_operand_map(&tmB, b_data, N, K, pair ? 128 : BN))
     return cudaErrorInvalidValue;
+  const auto* sa = static_cast<const uint8_t*>(a_scales);
+  const auto* sb = static_cast<const uint8_t*>(b_scales);
+  if (pair) {
+    static int max_pairs = -1;
+    if (max_pairs < 0) {
+      cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(P_SMEM_BYTES));
+      if (e != cudaSuccess) return e;
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(2 * (num_sms / 2));
+      q.blockDim = dim3(NUM_THREADS);
+      q.dynamicSmemBytes = P_SMEM_BYTES;
+      cudaLaunchAttribute qa[1];
+      qa[0].id = cudaLaunchAttributeClusterDimension;
+      qa[0].val.clusterDim.x = 2;
+      qa[0].val.clusterDim.y = 1;
+      qa[0].val.clusterDim.z = 1;
+      q.attrs = qa;
+      q.numAttrs = 1;
+      int n = 0;
+      e = cudaOccupancyMaxActiveClusters(&n, gemm_nvf4_pair_kernel, &q);
+      if (e != cudaSuccess || n < 1) n = num_sms / 2;
+      max_pairs = n;
+    }
+    const int64_t tiles = (M / 256) * (N / 256);
+    const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = P_SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel, tmA, tmB, sa, sb, a_gs, b_gs, static_cast<int>(M),
+                              static_cast<int>(N), static_cast<int>(K), D, out_bf16, ldd);
+  }
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -355,9 +655,8 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
   }
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-  gemm_nvf4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(
-      tmA, tmB, static_cast<const uint8_t*>(a_scales), static_cast<const uint8_t*>(b_scales), a_gs, b_gs,
-      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), D, out_bf16, ldd);
+  gemm_nvf4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(tmA, tmB, sa, sb, a_gs, b_gs, static_cast<int>(M),
+                                                         static_cast<int>(N), static_cast<int>(K), D, out_bf16, ldd);
   return cudaGetLastError();
 }
 

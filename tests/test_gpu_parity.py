@@ -182,6 +182,26 @@ def test_gemm_full_vs_oracle(M, N, K, bf16):
     assert_gemm_close(D.float().cpu().numpy(), D_ref, absum, bf16=bf16, what=f"gemm {M}x{N}x{K}")
 
 
+@pytest.mark.parametrize("M,N,K", [(256, 256, 256), (512, 768, 1280), (1024, 2048, 64), (768, 512, 320),
+                                   (2304, 1536, 512)])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_gemm_cta_pair_path_vs_oracle(M, N, K, bf16):
+    # M and N multiples of 256 take the CTA-pair kernel (cta_group::2)
+    xa = synth.activations(M, K, 63)
+    xb = synth.weights(N, K, 64, std=0.02)
+    qa, ca, sa, ga = _qrow(xa)
+    qb, cb, sb, gb = _qrow(xb)
+    D = api.gemm(qa, qb, api.OUT_BF16 if bf16 else api.OUT_F32)
+    if M * N <= 1 << 20:
+        D_ref, absum = O.gemm(ca, sa, ga, cb, sb, gb)
+        assert_gemm_close(D.float().cpu().numpy(), D_ref, absum, bf16=bf16, what=f"pair {M}x{N}x{K}")
+    else:
+        pairs = sample_pairs(M, N, 8192, seed=5)
+        D_ref, absum = O.gemm(ca, sa, ga, cb, sb, gb, pairs=pairs)
+        Dn = D.float().cpu().numpy()
+        assert_gemm_close(Dn[pairs[:, 0], pairs[:, 1]], D_ref, absum, bf16=bf16, what=f"pair {M}x{N}x{K}")
+
+
 def test_gemm_tiny_workload():
     x, w, _ = synth.workload_inputs("tiny")
     qa, ca, sa, ga = _qrow(x)
