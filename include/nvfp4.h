@@ -90,9 +90,10 @@ size_t nvfp4_scale_bytes(int64_t rows, int64_t cols);
  *   x         device BF16 [R, C], pitch ld >= C.
  *   rht       0: max |x|.  1: max |Q x| where Q = 1/4 * H16 * diag(s) acts on
  *             every aligned 16-run of rows of each column (section 2B.2; the
- *             amax of the tensor the Wgrad blocks are taken from).  Needs
- *             R % 16 == 0, C % 8 == 0, ld % 8 == 0.
- *   amax_dev  device, one float, overwritten (not accumulated).
+ *             amax of the tensor the Wgrad blocks are taken from).  2: both
+ *             from one pass over x: amax_dev[0] = max |x|, amax_dev[1] =
+ *             max |Q x|.  rht != 0 needs R % 16 == 0, C % 4 == 0, ld % 4 == 0.
+ *   amax_dev  device, one float (two for rht = 2), overwritten (not accumulated).
  */
 nvfp4_status nvfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht, float* amax_dev,
                         nvfp4_stream_t stream);

@@ -54,10 +54,11 @@ def empty_qtensor(rows, cols, device):
 
 
 def amax(x, rht=False, out=None):
-    """max|x| (rht=False) or max|Q x| along rows (rht=True) of a BF16 [R, C] tensor."""
+    """max|x| (rht=0), max|Q x| along rows (rht=1), or both from one pass
+    (rht=2: out[0] = max|x|, out[1] = max|Q x|) of a BF16 [R, C] tensor."""
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     if out is None:
-        out = torch.empty(1, dtype=torch.float32, device=x.device)
+        out = torch.empty(2 if int(rht) == 2 else 1, dtype=torch.float32, device=x.device)
     check("nvfp4_amax", lib().nvfp4_amax(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), int(rht),
                                          out.data_ptr(), _stream(x.device)))
     return out

@@ -85,28 +85,36 @@ __device__ __forceinline__ void fwht16(float (&v)[16]) {
 }
 
 // max |Q x| with Q = 1/4 * H16 * diag(s) on each aligned 16-run of rows of
-// every column.  Thread item: one 16-row band x 8 consecutive columns (sixteen
-// 16-byte loads, coalesced across the warp along the row).  The 1/4 is applied
+// every column (and, with BOTH, max |x| in the same pass).  Thread item: one
+// 16-row band x 4 consecutive columns: sixteen 8-byte loads, coalesced along
+// the row across the warp (256 bytes per row per warp).  The 1/4 is applied
 // after the maximum (an exact power-of-two scale commutes with max).
-__global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
-                                                         int64_t ld, uint32_t sign_mask,
-                                                         unsigned int* __restrict__ out) {
-  const int64_t groups = C / 8;
+template <bool BOTH>
+__global__ void __launch_bounds__(256, 3) amax_rht_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+                                                            int64_t ld, uint32_t sign_mask,
+                                                            unsigned int* __restrict__ out) {
+  const int64_t groups = C / 4;
   const int64_t items = (R / 16) * groups;
   float m = 0.0f;
+  uint32_t mplain = 0;
   for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items;
        it += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t band = it / groups, g = it - band * groups;
-    const uint16_t* base = x + band * 16 * ld + g * 8;
-    uint4 v[16];
+    const uint16_t* base = x + band * 16 * ld + g * 4;
+    uint2 v[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __ldcs(reinterpret_cast<const uint4*>(base + i * ld));
+    for (int i = 0; i < 16; ++i) v[i] = __ldcs(reinterpret_cast<const uint2*>(base + i * ld));
+    if (BOTH) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+      for (int i = 0; i < 16; ++i)
+        mplain = __vmaxu2(mplain, __vmaxu2(v[i].x & 0x7FFF7FFFu, v[i].y & 0x7FFF7FFFu));
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
       float f[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        uint32_t word = (c < 2) ? v[i].x : (c < 4) ? v[i].y : (c < 6) ? v[i].z : v[i].w;
+        const uint32_t word = (c < 2) ? v[i].x : v[i].y;
         uint32_t bits = (c & 1) ? (word >> 16) : (word & 0xFFFFu);
         bits ^= ((sign_mask >> i) & 1u) << 15;  // s_i = -1 flips the sign bit
         f[i] = bf16_bits_to_f32(bits);
@@ -117,30 +125,40 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
     }
   }
   m = __fmul_rn(m, 0.25f);
+  uint32_t mp = max(mplain & 0xFFFFu, mplain >> 16);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  if ((threadIdx.x & 31) == 0 && m > 0.0f) atomicMax(out, __float_as_uint(m));
+  for (int o = 16; o > 0; o >>= 1) {
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (BOTH) mp = max(mp, __shfl_xor_sync(0xFFFFFFFFu, mp, o));
+  }
+  if ((threadIdx.x & 31) == 0) {
+    if (m > 0.0f) atomicMax(out + (BOTH ? 1 : 0), __float_as_uint(m));
+    if (BOTH && mp) atomicMax(out, mp << 16);
+  }
 }
 
 cudaError_t launch_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht, uint32_t sign_mask,
                         float* amax_dev, int num_sms, cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(amax_dev, 0, sizeof(float), s);
+  cudaError_t e = cudaMemsetAsync(amax_dev, 0, (rht == 2 ? 2 : 1) * sizeof(float), s);
   if (e != cudaSuccess) return e;
   if (R == 0 || C == 0) return cudaSuccess;
   unsigned int* out = reinterpret_cast<unsigned int*>(amax_dev);
   if (rht) {
-    int64_t items = (R / 16) * (C / 8);
-    int64_t blocks = (items + 255) / 256;
-    int grid = static_cast<int>(blocks < 4LL * num_sms ? blocks : 4LL * num_sms);
-    amax_rht_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), R, C, ld, sign_mask, out);
+    const int64_t items = (R / 16) * (C / 4);
+    const int64_t blocks = (items + 255) / 256;
+    const int grid = static_cast<int>(blocks < 6LL * num_sms ? blocks : 6LL * num_sms);
+    if (rht == 2)
+      amax_rht_kernel<true><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), R, C, ld, sign_mask, out);
+    else
+      amax_rht_kernel<false><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), R, C, ld, sign_mask, out);
   } else if (ld == C && (R * C) % 8 == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
-    int64_t n8 = R * C / 8;
-    int64_t blocks = (n8 + 255) / 256;
-    int grid = static_cast<int>(blocks < 4LL * num_sms ? blocks : 4LL * num_sms);
+    const int64_t n8 = R * C / 8;
+    const int64_t blocks = (n8 + 255) / 256;
+    const int grid = static_cast<int>(blocks < 4LL * num_sms ? blocks : 4LL * num_sms);
     amax_flat_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), n8, out);
   } else {
-    int64_t blocks = (R + 7) / 8;
-    int grid = static_cast<int>(blocks < 8LL * num_sms ? blocks : 8LL * num_sms);
+    const int64_t blocks = (R + 7) / 8;
+    const int grid = static_cast<int>(blocks < 8LL * num_sms ? blocks : 8LL * num_sms);
     amax_rows_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), R, C, ld, out);
   }
   return cudaGetLastError();

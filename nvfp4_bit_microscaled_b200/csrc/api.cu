@@ -67,7 +67,8 @@ struct WsLayout {
   size_t total;
 };
 // Scalars at offset 0: amax slots (floats 0..7), decode scales (floats 8..15).
-enum { kAmaxX = 0, kAmaxW = 1, kAmaxXr = 2, kAmaxDy = 3, kAmaxDyr = 4 };
+// (kAmaxX, kAmaxXr) and (kAmaxDy, kAmaxDyr) are adjacent: one amax pass fills both.
+enum { kAmaxX = 0, kAmaxXr = 1, kAmaxW = 2, kAmaxDy = 3, kAmaxDyr = 4 };
 
 WsLayout ws_layout(int64_t T, int64_t Cin, int64_t Cout) {
   WsLayout L;
@@ -137,11 +138,11 @@ const char* nvfp4_status_string(nvfp4_status s) {
 
 nvfp4_status nvfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht, float* amax_dev,
                         nvfp4_stream_t stream) {
-  if (!x || !amax_dev) return NVFP4_ERR_INVALID_ARG;
+  if (!x || !amax_dev || rht < 0 || rht > 2) return NVFP4_ERR_INVALID_ARG;
   if (R < 0 || C < 0 || ld < C) return NVFP4_ERR_SHAPE;
   if (!aligned16(x) || (reinterpret_cast<uintptr_t>(amax_dev) & 3)) return NVFP4_ERR_ALIGN;
-  if (rht && (R % 16 || C % 8)) return NVFP4_ERR_SHAPE;
-  if (rht && ld % 8) return NVFP4_ERR_ALIGN;
+  if (rht && (R % 16 || C % 4)) return NVFP4_ERR_SHAPE;
+  if (rht && ld % 4) return NVFP4_ERR_ALIGN;
   DeviceInfo di;
   nvfp4_status st = device_info(&di);
   if (st != NVFP4_OK) return st;
@@ -234,7 +235,8 @@ nvfp4_status nvfp4_linear_fwd(const void* X, const void* W, int64_t T, int64_t C
   const nvfp4_tensor xr = ws_tensor(workspace, L, 0), wr = ws_tensor(workspace, L, 1),
                      wc = ws_tensor(workspace, L, 2), xc = ws_tensor(workspace, L, 3);
   // fprop operands: X row-wise (RN), W 2D (RN) with its transposed copy for dgrad
-  if ((st = nvfp4_amax(X, T, Cin, Cin, 0, amax + kAmaxX, stream)) != NVFP4_OK) return st;
+  // one pass over X gives both its amax (row copy) and its RHT amax (column copy)
+  if ((st = nvfp4_amax(X, T, Cin, Cin, 2, amax + kAmaxX, stream)) != NVFP4_OK) return st;
   if ((st = nvfp4_quantize(X, T, Cin, Cin, NVFP4_ROW, 0, 0, 0, amax + kAmaxX, &xr, nullptr, stream)) != NVFP4_OK)
     return st;
   if ((st = nvfp4_amax(W, Cout, Cin, Cin, 0, amax + kAmaxW, stream)) != NVFP4_OK) return st;
@@ -242,7 +244,6 @@ nvfp4_status nvfp4_linear_fwd(const void* X, const void* W, int64_t T, int64_t C
     return st;
   if ((st = nvfp4_gemm(&xr, &wr, Y, NVFP4_OUT_BF16, Cout, stream)) != NVFP4_OK) return st;
   // wgrad operand saved for the backward pass: X^T with the RHT along tokens (RN)
-  if ((st = nvfp4_amax(X, T, Cin, Cin, 1, amax + kAmaxXr, stream)) != NVFP4_OK) return st;
   return nvfp4_quantize(X, T, Cin, Cin, NVFP4_COL, 1, 0, 0, amax + kAmaxXr, nullptr, &xc, stream);
 }
 
@@ -257,13 +258,13 @@ nvfp4_status nvfp4_linear_bwd(const void* dY, int64_t T, int64_t Cin, int64_t Co
   const nvfp4_tensor wc = ws_tensor(workspace, L, 2), xc = ws_tensor(workspace, L, 3),
                      gr = ws_tensor(workspace, L, 4), gc = ws_tensor(workspace, L, 5);
   // dgrad: dX = dY W, dY row-wise with SR, W^T from the 2D column copy
-  if ((st = nvfp4_amax(dY, T, Cout, Cout, 0, amax + kAmaxDy, stream)) != NVFP4_OK) return st;
+  // one pass over dY gives both its amax (row copy) and its RHT amax (column copy)
+  if ((st = nvfp4_amax(dY, T, Cout, Cout, 2, amax + kAmaxDy, stream)) != NVFP4_OK) return st;
   if ((st = nvfp4_quantize(dY, T, Cout, Cout, NVFP4_ROW, 0, 1, seed, amax + kAmaxDy, &gr, nullptr, stream)) !=
       NVFP4_OK)
     return st;
   if ((st = nvfp4_gemm(&gr, &wc, dX, NVFP4_OUT_BF16, Cin, stream)) != NVFP4_OK) return st;
   // wgrad: dW = dY^T X, both with the RHT along tokens, SR on dY
-  if ((st = nvfp4_amax(dY, T, Cout, Cout, 1, amax + kAmaxDyr, stream)) != NVFP4_OK) return st;
   if ((st = nvfp4_quantize(dY, T, Cout, Cout, NVFP4_COL, 1, 1, seed, amax + kAmaxDyr, nullptr, &gc, stream)) !=
       NVFP4_OK)
     return st;

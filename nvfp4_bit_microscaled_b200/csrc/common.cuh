@@ -113,8 +113,11 @@ __host__ __device__ __forceinline__ u32x4 philox4x32_10(u32x4 c, uint32_t k0, ui
 #pragma unroll
   for (int round = 0; round < 10; ++round) {
 #if defined(__CUDA_ARCH__)
-    uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
-    uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+    uint32_t hi0, lo0, hi1, lo1;  // one 32x32 -> 64-bit multiply each
+    asm("{\n\t.reg .b64 p;\n\tmul.wide.u32 p, %2, 0xD2511F53;\n\tmov.b64 {%1, %0}, p;\n\t}"
+        : "=r"(hi0), "=r"(lo0) : "r"(c.x));
+    asm("{\n\t.reg .b64 p;\n\tmul.wide.u32 p, %2, 0xCD9E8D57;\n\tmov.b64 {%1, %0}, p;\n\t}"
+        : "=r"(hi1), "=r"(lo1) : "r"(c.z));
 #else
     uint64_t p0 = 0xD2511F53ull * c.x, p1 = 0xCD9E8D57ull * c.z;
     uint32_t hi0 = static_cast<uint32_t>(p0 >> 32), lo0 = static_cast<uint32_t>(p0);
@@ -138,19 +141,26 @@ __device__ __forceinline__ u32x4 sr_words(uint64_t g, uint32_t domain, uint32_t 
 
 // Stochastic rounding of a scaled value to the E2M1 grid: between the two
 // neighbouring grid magnitudes lo and lo + step, round up iff the 24-bit
-// uniform u = (w >> 8) * 2^-24 is below the fractional position p.  Grid steps
-// are 0.5 on [0,2), 1 on [2,4), 2 on [4,6]; all steps below are exact.
+// uniform u = (w >> 8) * 2^-24 is below the fractional position p.
 // ("Pretraining Large Language Models with NVFP4", section 2B.4 and the
 // "De Gok" example: 3.4 goes to 4 with probability 0.4.)
+//
+// On [1, 6] the E2M1 grid is the FP32 values with one mantissa bit, so p is
+// the 22 bits below it over 2^22, and u < p  <=>  (w >> 10) < frac22  <=>
+// frac22 + ((~w) >> 10) carries into that bit: add and truncate.  On [0.5, 1)
+// the grid is {0.5, 1} and the same holds with 23 bits and (~w) >> 9.  Below
+// 0.5 (grid {0, 0.5}, p = 2a) the comparison (w >> 8) < a * 2^25 is done in
+// FP32 (both sides exact).  Every case is the same decision as the
+// definition above, bit for bit.
 __device__ __forceinline__ float sr_magnitude(float y, uint32_t w) {
-  float a = fminf(fabsf(y), 6.0f);
-  float step = (a < 2.0f) ? 0.5f : ((a < 4.0f) ? 1.0f : 2.0f);
-  float inv = (a < 2.0f) ? 2.0f : ((a < 4.0f) ? 1.0f : 0.5f);
-  float lo = __fmul_rn(floorf(__fmul_rn(a, inv)), step);
-  float p = __fmul_rn(__fsub_rn(a, lo), inv);
-  float u = __fmul_rn(static_cast<float>(w >> 8), 5.9604644775390625e-08f);  // 2^-24
-  float mag = (u < p) ? __fadd_rn(lo, step) : lo;
-  return copysignf(mag, y);
+  const float a = fminf(fabsf(y), 6.0f);
+  const uint32_t b = __float_as_uint(a);
+  const bool big = a >= 1.0f;
+  const uint32_t keep = big ? 0xFFC00000u : 0xFF800000u;
+  const uint32_t rnd = (~w) >> (big ? 10 : 9);
+  const float upper = __uint_as_float((b + rnd) & keep);
+  const float lower = (__uint2float_rn(w >> 8) < __fmul_rn(a, 33554432.0f)) ? 0.5f : 0.0f;  // 2^25
+  return copysignf(a >= 0.5f ? upper : lower, y);
 }
 
 // --------------------------------------------------------------------------

@@ -57,7 +57,7 @@ __device__ __forceinline__ void fwht16(float (&v)[16]) {
 // Scale bytes of lanes 4j..4j+3 form one 32-bit word of the 128x4 tile layout.
 // ---------------------------------------------------------------------------
 template <bool SR>
-__global__ void __launch_bounds__(256, SR ? 3 : 4) quant_row_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+__global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
                                                           int64_t ld, const float* __restrict__ amax_dev,
                                                           uint32_t k0, uint32_t k1, uint8_t* __restrict__ data,
                                                           uint8_t* __restrict__ sf, int64_t sp,

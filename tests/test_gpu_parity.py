@@ -57,9 +57,14 @@ def test_amax_zero_tensor():
 def test_amax_rht_exact(name, x):
     R = x.shape[0] // 16 * 16
     x = x[:R].contiguous()
-    if x.shape[1] % 8:
-        pytest.skip("RHT amax needs C % 8 == 0")
     assert gpu_amax(x, rht=True) == O.amax_rht(x), name
+    both = api.amax(dev(x), rht=2).cpu().numpy()
+    assert both[0] == O.amax(x) and both[1] == O.amax_rht(x), name
+
+
+def test_amax_rht_narrow_columns():
+    x = synth.activations(48, 12, 33)            # C % 4 == 0 but C % 8 != 0
+    assert gpu_amax(x, rht=True) == O.amax_rht(x)
 
 
 # ------------------------------------------------------------------ row-wise
