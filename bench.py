@@ -352,51 +352,84 @@ def run_ours(args, rank, world, device):
 
 def run_e2e(args, rank, world, device, tensors):
     """Same metric through the public linear_fwd/linear_bwd calls with host
-    buffers: pinned host -> device copies of X, W, dY and device -> host copies
-    of Y, dX, dW inside the timed region."""
+    buffers: every step copies its X, W, dY from pinned host memory to the
+    device and its Y, dX, dW back to pinned host memory, inside the timed
+    region.  Copies run on their own streams and are pipelined across steps
+    (inputs of step i+1 and outputs of step i-1 move while step i computes),
+    with two device buffer sets; the data dependencies are kept by events."""
     X, W, dY = tensors
     T, Ci = X.shape
     Co = W.shape[0]
-    hX, hW, hdY = (t.cpu().pin_memory() for t in (X, W, dY))
-    hY = torch.empty(T, Co, dtype=torch.bfloat16).pin_memory()
-    hdX = torch.empty(T, Ci, dtype=torch.bfloat16).pin_memory()
-    hdW = torch.empty(Co, Ci, dtype=torch.float32).pin_memory()
-    dXd, dWd, dYd = torch.empty_like(X), torch.empty_like(W), torch.empty_like(dY)
-    ws = api.LinearWorkspace(T, Ci, Co, device)
-    Y = torch.empty(T, Co, dtype=torch.bfloat16, device=device)
-    gX = torch.empty(T, Ci, dtype=torch.bfloat16, device=device)
-    gW = torch.empty(Co, Ci, dtype=torch.float32, device=device)
+    steps = max(2, min(args.steps, 8))
+    hin = [tuple(t.cpu().pin_memory() for t in (X, W, dY)) for _ in range(2)]
+    hout = [(torch.empty(T, Co, dtype=torch.bfloat16).pin_memory(),
+             torch.empty(T, Ci, dtype=torch.bfloat16).pin_memory(),
+             torch.empty(Co, Ci, dtype=torch.float32).pin_memory()) for _ in range(2)]
+    din = [(torch.empty_like(X), torch.empty_like(W), torch.empty_like(dY)) for _ in range(2)]
+    dout = [(torch.empty(T, Co, dtype=torch.bfloat16, device=device), torch.empty(T, Ci, dtype=torch.bfloat16, device=device),
+             torch.empty(Co, Ci, dtype=torch.float32, device=device)) for _ in range(2)]
+    ws = [api.LinearWorkspace(T, Ci, Co, device) for _ in range(2)]
+    compute, h2d, d2h = torch.cuda.current_stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
-    def one():
-        dXd.copy_(hX, non_blocking=True)
-        dWd.copy_(hW, non_blocking=True)
-        dYd.copy_(hdY, non_blocking=True)
-        api.linear_fwd(dXd, dWd, ws, Y=Y)
-        api.linear_bwd(dYd, ws, WORKLOAD["sr_seed"], dX=gX, dW=gW)
-        hY.copy_(Y, non_blocking=True)
-        hdX.copy_(gX, non_blocking=True)
-        hdW.copy_(gW, non_blocking=True)
+    def run(n):
+        loaded = [None, None]      # event: inputs of buffer b on the device
+        computed = [None, None]    # event: outputs of buffer b ready
+        drained = [None, None]     # event: outputs of buffer b copied out (buffer b reusable)
+        consumed = [None, None]    # event: inputs of buffer b no longer needed
+        def load(i):
+            b = i % 2
+            with torch.cuda.stream(h2d):
+                if consumed[b] is not None:
+                    h2d.wait_event(consumed[b])
+                for d, h in zip(din[b], hin[b]):
+                    d.copy_(h, non_blocking=True)
+                loaded[b] = torch.cuda.Event()
+                loaded[b].record(h2d)
+        load(0)
+        for i in range(n):
+            b = i % 2
+            if i + 1 < n:
+                load(i + 1)
+            compute.wait_event(loaded[b])
+            if drained[b] is not None:
+                compute.wait_event(drained[b])
+            Xd, Wd, Gd = din[b]
+            Y, gX, gW = dout[b]
+            api.linear_fwd(Xd, Wd, ws[b], Y=Y)
+            api.linear_bwd(Gd, ws[b], WORKLOAD["sr_seed"], dX=gX, dW=gW)
+            consumed[b] = torch.cuda.Event()
+            consumed[b].record(compute)
+            computed[b] = torch.cuda.Event()
+            computed[b].record(compute)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(computed[b])
+                for h, d in zip(hout[b], dout[b]):
+                    h.copy_(d, non_blocking=True)
+                drained[b] = torch.cuda.Event()
+                drained[b].record(d2h)
+        compute.wait_event(drained[(n - 1) % 2])
+        if n > 1:
+            compute.wait_event(drained[(n - 2) % 2])
 
-    steps = max(1, min(args.steps, 5))
-    for _ in range(min(args.warmup, 2)):
-        one()
+    run(2)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(steps):
-        one()
-    e.record()
+    s.record(compute)
+    h2d.wait_event(s)
+    d2h.wait_event(s)
+    run(steps)
+    e.record(compute)
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e), device, world)
     ms_step = ms / steps
     flops = 3 * 2.0 * T * Ci * Co
-    h2d = sum(t.numel() * t.element_size() for t in (hX, hW, hdY))
-    d2h = sum(t.numel() * t.element_size() for t in (hY, hdX, hdW))
+    h2d_b = sum(t.numel() * t.element_size() for t in hin[0])
+    d2h_b = sum(t.numel() * t.element_size() for t in hout[0])
     return {"value": round(flops * world / (ms_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_step, 3),
-            "steps": steps}
+            "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b, "ms_per_step": round(ms_step, 3),
+            "steps": steps, "pipelined": "H2D of step i+1 and D2H of step i-1 overlap step i (copy streams)"}
 
 
 # --------------------------------------------------------------------------- reference arm
