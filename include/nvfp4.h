@@ -207,6 +207,12 @@ uint32_t nvfp4_rht_sign_mask(void);
 const char* nvfp4_status_string(nvfp4_status status);
 int nvfp4_version(void);
 
+/* The cudaError_t code behind the most recent NVFP4_ERR_CUDA returned to this
+ * host thread (0 if none yet); *name, when name is not NULL, receives the
+ * CUDA runtime's name for it (a static string).  Library bookkeeping only:
+ * the pages define no such call. */
+int nvfp4_last_cuda_error(const char** name);
+
 #ifdef __cplusplus
 }
 #endif

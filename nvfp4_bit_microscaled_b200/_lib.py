@@ -10,6 +10,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
 
 NVFP4_OK = 0
+NVFP4_ERR_CUDA = 6
 STATUS_NAMES = {
     0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_SHAPE", 3: "NVFP4_ERR_ALIGN",
     4: "NVFP4_ERR_UNSUPPORTED", 5: "NVFP4_ERR_DEVICE", 6: "NVFP4_ERR_CUDA", 7: "NVFP4_ERR_WORKSPACE",
@@ -25,9 +26,11 @@ class Nvfp4Tensor(ctypes.Structure):
 
 
 class Nvfp4Error(RuntimeError):
-    def __init__(self, fn, status):
+    def __init__(self, fn, status, cuda_error=None):
         self.status = status
-        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+        self.cuda_error = cuda_error
+        extra = f" ({cuda_error[1]}, code {cuda_error[0]})" if cuda_error else ""
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}{extra}")
 
 
 _c = ctypes
@@ -50,6 +53,7 @@ PROTOTYPES = {
     "nvfp4_rht_sign_mask": (_u32, []),
     "nvfp4_status_string": (_c.c_char_p, [_int]),
     "nvfp4_version": (_int, []),
+    "nvfp4_last_cuda_error": (_int, [_c.POINTER(_c.c_char_p)]),
 }
 
 _LIB = None
@@ -74,4 +78,9 @@ def lib():
 
 def check(fn_name, status):
     if status != NVFP4_OK:
-        raise Nvfp4Error(fn_name, status)
+        cuda_error = None
+        if status == NVFP4_ERR_CUDA and _LIB is not None:
+            name = _c.c_char_p()
+            code = _LIB.nvfp4_last_cuda_error(_c.byref(name))
+            cuda_error = (code, (name.value or b"?").decode())
+        raise Nvfp4Error(fn_name, status, cuda_error)

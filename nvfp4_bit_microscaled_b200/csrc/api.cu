@@ -44,7 +44,14 @@ nvfp4_status device_info(DeviceInfo* out) {
   return NVFP4_OK;
 }
 
-inline nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+// Last CUDA error code behind an NVFP4_ERR_CUDA, per host thread.
+thread_local int t_last_cuda_error = 0;
+
+inline nvfp4_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return NVFP4_OK;
+  t_last_cuda_error = static_cast<int>(e);
+  return NVFP4_ERR_CUDA;
+}
 
 uint32_t sign_mask() {
   const nvfp4::u32x4 w = nvfp4::philox4x32_10(nvfp4::u32x4{0u, 0u, nvfp4::kDomainRhtSigns, 0u}, 0u, 0u);
@@ -121,6 +128,12 @@ uint32_t nvfp4_rht_sign_mask(void) { return sign_mask(); }
 
 int nvfp4_version(void) { return 1; }
 
+int nvfp4_last_cuda_error(const char** name) {
+  const int e = t_last_cuda_error;
+  if (name) *name = cudaGetErrorName(static_cast<cudaError_t>(e));
+  return e;
+}
+
 const char* nvfp4_status_string(nvfp4_status s) {
   switch (s) {
     case NVFP4_OK: return "ok";
@@ -183,12 +196,12 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, nvf
   if (want_row) {
     e = nvfp4::launch_quant_row(x, R, C, ld, amax_dev, sr, seed, row_out->data, row_out->scales,
                                 row_out->global_scale, di.sms, s);
-    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
   }
   if (want_col) {
     e = nvfp4::launch_quant_col(x, R, C, ld, amax_dev, rht, sign_mask(), sr, seed, col_out->data,
                                 col_out->scales, col_out->global_scale, di.sms, s);
-    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
   }
   return NVFP4_OK;
 }

@@ -324,6 +324,16 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 // reads B's scales from each CTA.  The leader (cluster rank 0) issues the
 // MMAs; both CTAs' loads, scale writes and epilogues report to the leader's
 // barriers, and the leader's commits arrive in both CTAs.
+//
+// The epilogue writes the output through shared memory and TMA stores (one
+// 32-row x 128-byte box per warp at a time, 128-byte swizzle), not with
+// per-thread global stores: those touch 32 rows per warp instruction and flood
+// the SM's load/store queue, which the barrier waits, the scale warps and the
+// MMA issuer also go through, so the next tile's pipeline stalls behind them
+// (measured: 5-16 thousand cycles per tile boundary).  For the same reason the
+// MMA issuer does nothing between the four MMAs of a stage: every extra
+// instruction there, even a non-blocking barrier probe, showed up as idle
+// tensor-pipe time.
 // ===========================================================================
 constexpr int P_STAGES = 5;
 constexpr uint32_t P_A_BYTES = 128 * BK_BYTES;                 // 16 KiB (own A rows)
@@ -334,8 +344,12 @@ constexpr uint32_t P_OFF_A = 0;
 constexpr uint32_t P_OFF_B = P_OFF_A + P_STAGES * P_A_BYTES;
 constexpr uint32_t P_OFF_SFA = P_OFF_B + P_STAGES * P_B_BYTES;
 constexpr uint32_t P_OFF_SFB = P_OFF_SFA + P_STAGES * P_SFA_BYTES;
-constexpr uint32_t P_OFF_BAR = P_OFF_SFB + P_STAGES * P_SFB_BYTES;
+constexpr uint32_t P_STG_BYTES = 32 * 128;                     // one 32-row x 128-byte output box per epilogue warp
+constexpr uint32_t P_OFF_STG = P_OFF_SFB + P_STAGES * P_SFB_BYTES;
+constexpr uint32_t P_OFF_BAR = P_OFF_STG + NUM_EPI_WARPS * P_STG_BYTES;
 constexpr uint32_t P_SMEM_BYTES = P_OFF_BAR + 512 + 1024;
+static_assert(P_OFF_STG % 1024 == 0, "swizzled staging boxes need 1024-byte alignment");
+static_assert(P_SMEM_BYTES <= 232448, "pair kernel shared memory exceeds the per-block limit");
 constexpr int P_GROUP_M = 8;
 
 // kind::mxf4nvf4, A/B E2M1 K-major, UE4M3 scales, M = 256 (pair), N = 256.
@@ -345,9 +359,9 @@ __host__ __device__ constexpr uint32_t make_idesc_pair() {
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
-                      const float* __restrict__ gsa, const float* __restrict__ gsb, int M, int N, int K,
-                      void* __restrict__ D, int out_bf16, int64_t ldd) {
+                      const __grid_constant__ CUtensorMap tmD, const uint8_t* __restrict__ sfa,
+                      const uint8_t* __restrict__ sfb, const float* __restrict__ gsa,
+                      const float* __restrict__ gsb, int M, int N, int K, int out_bf16) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_OFF_BAR);   // leader: A/B bytes of both CTAs
@@ -382,6 +396,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     fence_barrier_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmD);
   }
   if (warp == 1) tmem_alloc_pair(const_cast<uint32_t*>(tmem_slot), TMEM_COLS);
   tc_fence_before();
@@ -438,6 +453,9 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     uint32_t phase = 0, acc_phase = 0;
     const uint32_t a_base = smem_u32(smem + P_OFF_A), b_base = smem_u32(smem + P_OFF_B);
     const uint32_t idesc = make_idesc_pair();
+    // Stage descriptors differ only in the start-address field (address >> 4,
+    // bits 0-13): adding stage * bytes / 16 moves to the stage's tile.
+    const uint64_t adesc0 = smem_desc(a_base, 16, 1024, 2), bdesc0 = smem_desc(b_base, 16, 1024, 2);
     for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
       if (!mbar_wait_cluster(acc_empty, acc_phase ^ 1u, kErrWaitAccEmpty)) { *abort_flag = 1; break; }
       tc_fence_after();
@@ -450,13 +468,21 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
           break;
         }
         tc_fence_after();
-        const int nkb = min(KB_PER_STAGE, katoms - kt * KB_PER_STAGE);
         const uint32_t sfa_t = tmem + SF_COL + stage * SF_BUF_COLS, sfb_t = sfa_t + SFB_OFF;
-        const uint64_t adesc = smem_desc(a_base + stage * P_A_BYTES, 16, 1024, 2);
-        const uint64_t bdesc = smem_desc(b_base + stage * P_B_BYTES, 16, 1024, 2);
-        for (int kb = 0; kb < nkb; ++kb)
-          mma_nvf4_pair(tmem + ACC_COL, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa_t + 4 * kb, sfb_t + 8 * kb,
-                        (kt | kb) != 0);
+        const uint64_t adesc = adesc0 + static_cast<uint64_t>(stage * (P_A_BYTES >> 4));
+        const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(stage * (P_B_BYTES >> 4));
+        if ((kt + 1) * KB_PER_STAGE <= katoms) {
+          // full stage: four MMAs back to back, nothing else between them
+#pragma unroll
+          for (int kb = 0; kb < KB_PER_STAGE; ++kb)
+            mma_nvf4_pair(tmem + ACC_COL, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa_t + 4 * kb, sfb_t + 8 * kb,
+                          (kt | kb) != 0);
+        } else {
+          const int nkb = katoms - kt * KB_PER_STAGE;
+          for (int kb = 0; kb < nkb; ++kb)
+            mma_nvf4_pair(tmem + ACC_COL, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa_t + 4 * kb, sfb_t + 8 * kb,
+                          (kt | kb) != 0);
+        }
         tc_commit_pair_mc(&empty[stage], 0x3);
         if (++stage == P_STAGES) stage = 0, phase ^= 1u;
       }
@@ -506,10 +532,19 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     }
   } else if (warp >= EPI_WARP0) {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    // Warp w reads TMEM lanes 32*(w%4) .. +31 (its rows) and 128 accumulator
+    // columns, scales by alpha, and stores 32-row x 128-byte boxes (64 BF16 or
+    // 32 FP32 columns) through its staging buffer: row r's 16-byte chunk j
+    // sits at r*128 + 16*(j ^ (r%8)), the 128-byte swizzle the output tensor
+    // map names, so the eight lanes that write one 128-byte row band hit
+    // distinct bank groups.
     const int quarter = warp & 3;
     const int col_half = (warp - EPI_WARP0) >> 2;
     const float alpha = __fmul_rn(__ldg(gsa), __ldg(gsb));
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    uint8_t* stg = smem + P_OFF_STG + (warp - EPI_WARP0) * P_STG_BYTES;
+    uint8_t* my_row = stg + lane * 128;
+    const int sw = lane & 7;
     uint32_t acc_phase = 0;
     for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
       const int per_group = P_GROUP_M * num_n, grp = t / per_group, first_m = grp * P_GROUP_M;
@@ -517,49 +552,72 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
       const int tm = first_m + within % gsize, tn = within / gsize;
       if (!mbar_wait_cluster(acc_full, acc_phase, kErrWaitAccFull)) { *abort_flag = 1; break; }
       tc_fence_after();
-      const int row = tm * 256 + 128 * static_cast<int>(rank) + quarter * 32 + lane;
+      const int row0 = tm * 256 + 128 * static_cast<int>(rank) + quarter * 32;
       const int col_base = tn * 256 + col_half * 128;
       if (out_bf16) {
-        uint32_t packed[64];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + ACC_COL + col_half * 128 + ch * 32, r);
-          tmem_ld_wait();
+        for (int h = 0; h < 2; ++h) {  // two boxes of 64 columns
+          uint32_t packed[32];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
-                                                     __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
-            packed[16 * ch + e] = *reinterpret_cast<uint32_t*>(&h);
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(tmem + lane_base + ACC_COL + col_half * 128 + h * 64 + ch * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              __nv_bfloat162 v = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
+                                                       __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
+              packed[16 * ch + e] = *reinterpret_cast<uint32_t*>(&v);
+            }
+          }
+          if (h == 1) {  // every accumulator column of this warp is in registers
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_l);
+          }
+          if (lane == 0) bulk_wait_read_all();  // the previous box has left the staging buffer
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(my_row + 16 * (j ^ sw)) =
+                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmD, stg, col_base + 64 * h, row0);
+            bulk_commit_group();
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(acc_empty_l);
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(D) + static_cast<int64_t>(row) * ldd + col_base;
-#pragma unroll
-        for (int v = 0; v < 16; ++v)
-          reinterpret_cast<uint4*>(dst)[v] =
-              make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
       } else {
-        for (int ch = 0; ch < 4; ++ch) {
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {  // four boxes of 32 columns
           uint32_t r[32];
           tmem_ld_32x32b_x32(tmem + lane_base + ACC_COL + col_half * 128 + ch * 32, r);
           tmem_ld_wait();
-          float* dst = static_cast<float*>(D) + static_cast<int64_t>(row) * ldd + col_base + ch * 32;
+          if (ch == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_l);
+          }
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            reinterpret_cast<float4*>(dst)[v] = make_float4(__fmul_rn(__uint_as_float(r[4 * v + 0]), alpha),
-                                                            __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
-                                                            __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha),
-                                                            __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4*>(my_row + 16 * (j ^ sw)) = make_float4(
+                __fmul_rn(__uint_as_float(r[4 * j + 0]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 1]), alpha),
+                __fmul_rn(__uint_as_float(r[4 * j + 2]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 3]), alpha));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmD, stg, col_base + 32 * ch, row0);
+            bulk_commit_group();
+          }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(acc_empty_l);
       }
       acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_all();  // stores complete before the CTA (and its shared memory) goes away
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -596,15 +654,36 @@ bool make_operand_map(CUtensorMap* tm, const void* data, int64_t rows, int64_t K
   return r == CUDA_SUCCESS;
 }
 
+// Output D [M, N] (row stride ldd elements), stored in 32-row x 128-byte boxes
+// (64 BF16 or 32 FP32 columns) from 128-byte-swizzled shared memory.
+bool make_output_map(CUtensorMap* tm, void* D, int64_t M, int64_t N, int64_t ldd, int out_bf16) {
+  auto encode = get_encode_fn();
+  if (!encode) return false;
+  const int64_t esize = out_bf16 ? 2 : 4;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldd * esize)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(tm, out_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, D, dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a_gs, const void* b_data,
                         const void* b_scales, const float* b_gs, int64_t M, int64_t N, int64_t K, void* D,
                         int out_bf16, int64_t ldd, int num_sms, cudaStream_t s) {
-  const bool pair = (M % 256 == 0) && (N % 256 == 0);
-  CUtensorMap tmA, tmB;
+  // The pair kernel stores through TMA: the output base must be 16-byte
+  // aligned and its row stride a multiple of 16 bytes.
+  const int64_t esize = out_bf16 ? 2 : 4;
+  const bool pair = (M % 256 == 0) && (N % 256 == 0) && (reinterpret_cast<uintptr_t>(D) % 16 == 0) &&
+                    ((ldd * esize) % 16 == 0);
+  CUtensorMap tmA, tmB, tmD;
   if (!make_operand_map(&tmA, a_data, M, K, BM) || !make_operand_map(&tmB, b_data, N, K, pair ? 128 : BN))
     return cudaErrorInvalidValue;
+  if (pair && !make_output_map(&tmD, D, M, N, ldd, out_bf16)) return cudaErrorInvalidValue;
   const auto* sa = static_cast<const uint8_t*>(a_scales);
   const auto* sb = static_cast<const uint8_t*>(b_scales);
   if (pair) {
@@ -643,8 +722,8 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel, tmA, tmB, sa, sb, a_gs, b_gs, static_cast<int>(M),
-                              static_cast<int>(N), static_cast<int>(K), D, out_bf16, ldd);
+    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel, tmA, tmB, tmD, sa, sb, a_gs, b_gs, static_cast<int>(M),
+                              static_cast<int>(N), static_cast<int>(K), out_bf16);
   }
   static bool attr_set = false;
   if (!attr_set) {

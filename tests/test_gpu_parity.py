@@ -6,6 +6,7 @@ import torch
 
 import oracle as O
 from nvfp4_bit_microscaled_b200 import api, synth
+from nvfp4_bit_microscaled_b200._lib import Nvfp4Error
 from tests._parity import assert_gemm_close, assert_q_equal, dev, gpu_amax, sample_pairs
 
 pytestmark = pytest.mark.gpu
@@ -205,6 +206,36 @@ def test_gemm_cta_pair_path_vs_oracle(M, N, K, bf16):
         D_ref, absum = O.gemm(ca, sa, ga, cb, sb, gb, pairs=pairs)
         Dn = D.float().cpu().numpy()
         assert_gemm_close(Dn[pairs[:, 0], pairs[:, 1]], D_ref, absum, bf16=bf16, what=f"pair {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("pad", [8, 24])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_gemm_output_row_stride(pad, bf16):
+    # D written into a wider buffer (row stride N + pad) by the CTA-pair
+    # kernel's TMA-store epilogue; the columns past N stay untouched.
+    M, N, K = 512, 256, 320
+    xa = synth.activations(M, K, 65)
+    xb = synth.weights(N, K, 66, std=0.02)
+    qa, ca, sa, ga = _qrow(xa)
+    qb, cb, sb, gb = _qrow(xb)
+    dt = torch.bfloat16 if bf16 else torch.float32
+    buf = torch.full((M, N + pad), 7.0, dtype=dt, device="cuda")
+    api.gemm(qa, qb, api.OUT_BF16 if bf16 else api.OUT_F32, out=buf[:, :N])
+    D_ref, absum = O.gemm(ca, sa, ga, cb, sb, gb)
+    got = buf.float().cpu().numpy()
+    assert_gemm_close(got[:, :N], D_ref, absum, bf16=bf16, what=f"ldd {N + pad}")
+    assert (got[:, N:] == 7.0).all()
+
+
+def test_gemm_rejects_unaligned_row_stride_before_launch():
+    M, N, K = 256, 256, 64
+    qa, _, _, _ = _qrow(synth.activations(M, K, 67))
+    qb, _, _, _ = _qrow(synth.weights(N, K, 68, std=0.02))
+    buf = torch.zeros((M, N + 3), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(Nvfp4Error) as e:
+        api.gemm(qa, qb, api.OUT_BF16, out=buf[:, :N])
+    assert e.value.status == 3  # NVFP4_ERR_ALIGN
+    assert (buf == 0).all()
 
 
 def test_gemm_tiny_workload():

@@ -55,6 +55,13 @@ def test_status_strings(L):
         assert L.nvfp4_status_string(k)
 
 
+def test_last_cuda_error_starts_clear(L):
+    name = ctypes.c_char_p()
+    assert L.nvfp4_last_cuda_error(None) == 0
+    assert L.nvfp4_last_cuda_error(ctypes.byref(name)) == 0
+    assert name.value == b"cudaSuccess"
+
+
 def _t(rows, cols, data=4096, scales=8192, gs=16384):
     return _lib.Nvfp4Tensor(data, scales, gs, rows, cols)
 
