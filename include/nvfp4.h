@@ -204,6 +204,15 @@ nvfp4_status nvfp4_wait_probe(uint32_t timeout_us, nvfp4_stream_t stream);
  * of Philox4x32-10 with key 0 and counter (0, 0, 2, 0). */
 uint32_t nvfp4_rht_sign_mask(void);
 
+/* Self-test of the block-scale arithmetic: the kernels compute d / 6 (the
+ * E4M3 scale of section 2A) with a multiply and two fma's instead of an IEEE
+ * division.  This runs both on every non-negative finite float and reports
+ * how many quotients differ where the IEEE quotient is a normal float
+ * (*bad_quotients) and how many E4M3 codes differ at all (*bad_codes); both
+ * must be 0.  Synchronous, on the current device.  Library bookkeeping: the
+ * pages define no such call. */
+nvfp4_status nvfp4_selftest_scale_division(uint64_t* bad_quotients, uint64_t* bad_codes);
+
 const char* nvfp4_status_string(nvfp4_status status);
 int nvfp4_version(void);
 

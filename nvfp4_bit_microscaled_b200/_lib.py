@@ -54,6 +54,7 @@ PROTOTYPES = {
     "nvfp4_status_string": (_c.c_char_p, [_int]),
     "nvfp4_version": (_int, []),
     "nvfp4_last_cuda_error": (_int, [_c.POINTER(_c.c_char_p)]),
+    "nvfp4_selftest_scale_division": (_int, [_c.POINTER(_c.c_uint64), _c.POINTER(_c.c_uint64)]),
 }
 
 _LIB = None

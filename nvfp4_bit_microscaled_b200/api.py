@@ -152,3 +152,12 @@ def read_device_error(clear=True):
 
 def wait_probe(timeout_us, device=None):
     check("nvfp4_wait_probe", lib().nvfp4_wait_probe(int(timeout_us), _stream(device)))
+
+
+def selftest_scale_division():
+    """(bad_quotients, bad_codes) of the kernels' divide-by-6 against IEEE division on every
+    non-negative finite float; both are 0 on a correct build."""
+    q, c = ctypes.c_uint64(0), ctypes.c_uint64(0)
+    check("nvfp4_selftest_scale_division",
+          lib().nvfp4_selftest_scale_division(ctypes.byref(q), ctypes.byref(c)))
+    return q.value, c.value

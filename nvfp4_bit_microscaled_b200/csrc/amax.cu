@@ -97,9 +97,16 @@ __global__ void __launch_bounds__(256, 3) amax_rht_kernel(const uint16_t* __rest
   const int64_t items = (R / 16) * groups;
   float m = 0.0f;
   uint32_t mplain = 0;
-  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items;
-       it += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t band = it / groups, g = it - band * groups;
+  // item it = (band it / groups, column group it % groups), kept incrementally
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x, step_q = step / groups,
+                step_r = step - step_q * groups;
+  int64_t band_next = first / groups, g_next = first - band_next * groups;
+  for (int64_t it = first; it < items; it += step) {
+    const int64_t band = band_next, g = g_next;
+    g_next += step_r;
+    band_next += step_q;
+    if (g_next >= groups) g_next -= groups, ++band_next;
     const uint16_t* base = x + band * 16 * ld + g * 4;
     uint2 v[16];
 #pragma unroll

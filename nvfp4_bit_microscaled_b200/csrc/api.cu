@@ -126,6 +126,18 @@ size_t nvfp4_scale_bytes(int64_t rows, int64_t cols) {
 
 uint32_t nvfp4_rht_sign_mask(void) { return sign_mask(); }
 
+nvfp4_status nvfp4_selftest_scale_division(uint64_t* bad_quotients, uint64_t* bad_codes) {
+  if (!bad_quotients || !bad_codes) return NVFP4_ERR_INVALID_ARG;
+  DeviceInfo di;
+  nvfp4_status st = device_info(&di);
+  if (st != NVFP4_OK) return st;
+  unsigned long long q = 0, c = 0;
+  st = cuda_status(nvfp4::selftest_div6(&q, &c, di.sms));
+  *bad_quotients = q;
+  *bad_codes = c;
+  return st;
+}
+
 int nvfp4_version(void) { return 1; }
 
 int nvfp4_last_cuda_error(const char** name) {

@@ -189,6 +189,44 @@ __device__ __forceinline__ BlockScale block_scale(float bamax, float s_enc) {
   return b;
 }
 
+// x / 6 rounded to nearest-even, for finite x >= 0, by one correction step of
+// a reciprocal product (Markstein, "Computation of elementary functions on the
+// IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): q = x*c with
+// c = RN(1/6), the remainder x - 6q is exact in one fma, and q + rem*c is
+// within a tiny fraction of an ulp of x/6.  x/6 = (x/3)/2 and x/3 is never
+// closer than ulp/6 to a rounding midpoint (3 does not divide a power of two),
+// so that last fma rounds to the same float as the exact quotient.  Where the
+// quotient is an FP32 subnormal the two may differ in the last place; those
+// values are far below the smallest E4M3 scale (2^-9), whose encoding is 0
+// either way.  A self-test compares it with the IEEE division on every
+// non-negative float.
+__device__ __forceinline__ float div6_rn(float x) {
+  const float c = 0.166666672f;  // RN(1/6) = 0x3E2AAAAB
+  const float q = __fmul_rn(x, c);
+  const float rem = __fmaf_rn(-q, 6.0f, x);
+  return __fmaf_rn(rem, c, q);
+}
+
+// r = S_enc / s_b for every E4M3 code (0 where the code decodes to 0): one
+// IEEE division per code, done once per CTA into shared memory, so a block
+// scale costs a table load instead of a division.  Codes 0x7F and above never
+// occur (the encode saturates at 0x7E = 448).
+constexpr int kRTableSize = 128;
+__device__ __forceinline__ void fill_r_table(float* tbl, float s_enc) {
+  for (int j = threadIdx.x; j < kRTableSize; j += blockDim.x) {
+    const float sb = e4m3_to_f32(static_cast<uint32_t>(j));
+    tbl[j] = (sb == 0.0f) ? 0.0f : __fdiv_rn(s_enc, sb);
+  }
+}
+
+// block_scale() with the divisions above: the same scale byte and r, bit for bit.
+__device__ __forceinline__ BlockScale block_scale_t(float bamax, float s_enc, const float* r_tbl) {
+  BlockScale b;
+  b.sf = f32_to_e4m3(div6_rn(__fmul_rn(bamax, s_enc)));
+  b.r = r_tbl[b.sf];
+  return b;
+}
+
 // --------------------------------------------------------------------------
 // Scale-factor layout: 128x4 tiles of 512 bytes, the block-scale layout the
 // tensor core's block-scaled MMA reads (one tile = 128 rows x 4 scales).

@@ -25,6 +25,10 @@ cudaError_t launch_quant_2d(const void* w, int64_t N, int64_t K, int64_t ld, con
                             void* row_data, void* row_scales, float* row_gs, void* col_data, void* col_scales,
                             float* col_gs, int num_sms, cudaStream_t s);
 
+// Self-test: the block-scale divide-by-6 against the IEEE division on every
+// non-negative finite float (synchronous, default stream).
+cudaError_t selftest_div6(unsigned long long* bad_quotients, unsigned long long* bad_codes, int num_sms);
+
 // Zero the padding of a scale matrix (rows >= R or scale columns >= S).
 cudaError_t launch_sf_pad_zero(void* scales, int64_t R, int64_t S, cudaStream_t s);
 

@@ -63,26 +63,42 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
                                                           uint8_t* __restrict__ sf, int64_t sp,
                                                           float* __restrict__ gs_out) {
   constexpr int U = SR ? 1 : 2;  // items in flight per warp
+  __shared__ float r_tbl[kRTableSize];
   const float amax = __ldg(amax_dev);
   const float s_enc = encode_scale(amax);
   if (blockIdx.x == 0 && threadIdx.x == 0 && gs_out) *gs_out = decode_scale(amax);
+  fill_r_table(r_tbl, s_enc);
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int64_t S = C >> 4;
   const int64_t nseg = (S + 31) >> 5;
   const int64_t items = R * nseg;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int64_t half_c = C >> 1;
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  // item it = (row it / nseg, segment it % nseg), kept incrementally: one
+  // division per thread instead of one per item
+  const int64_t step = U * nwarps, step_q = step / nseg, step_r = step - step_q * nseg;
+  int64_t row_u[U], seg_u[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int64_t it = first + u * nwarps;
+    row_u[u] = it / nseg;
+    seg_u[u] = it - row_u[u] * nseg;
+  }
 
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); base < items;
-       base += U * nwarps) {
+  for (int64_t base = first; base < items; base += step) {
     uint4 v[U][2];
     int64_t rr[U], bb[U];
     bool ok[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int64_t it = base + u * nwarps;
-      const int64_t r = it / nseg;
-      const int64_t b = (it - r * nseg) * 32 + lane;
+      const int64_t r = row_u[u];
+      const int64_t b = seg_u[u] * 32 + lane;
+      seg_u[u] += step_r;
+      row_u[u] += step_q;
+      if (seg_u[u] >= nseg) seg_u[u] -= nseg, ++row_u[u];
       rr[u] = r;
       bb[u] = b;
       ok[u] = (it < items) && (b < S);
@@ -97,7 +113,7 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
     for (int u = 0; u < U; ++u) {
       if (base + u * nwarps >= items) break;  // warp-uniform
       const uint32_t mb = max(absmax_bits8(v[u][0]), absmax_bits8(v[u][1]));
-      const BlockScale bs = block_scale(bf16_bits_to_f32(mb), s_enc);
+      const BlockScale bs = block_scale_t(bf16_bits_to_f32(mb), s_enc, r_tbl);
       float y[16];
       unpack8(v[u][0], y);
       unpack8(v[u][1], y + 8);
@@ -141,18 +157,27 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
                                                              uint32_t sign_mask, uint32_t k0, uint32_t k1,
                                                              uint8_t* __restrict__ data, uint8_t* __restrict__ sf,
                                                              int64_t sp, float* __restrict__ gs_out) {
+  __shared__ float r_tbl[kRTableSize];
   const float amax = __ldg(amax_dev);
   const float s_enc = encode_scale(amax);
   if (blockIdx.x == 0 && threadIdx.x == 0 && gs_out) *gs_out = decode_scale(amax);
+  fill_r_table(r_tbl, s_enc);
+  __syncthreads();
   const int64_t S = R >> 4;
   const int64_t nq = (S + 3) >> 2;
   const int64_t ng = C >> 2;
   const int64_t items = nq * ng;
   const int64_t half_r = R >> 1;
+  // item it = (token quad it / ng, channel group it % ng), kept incrementally
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x, step_q = step / ng, step_r = step - step_q * ng;
+  int64_t q_next = first / ng, g_next = first - q_next * ng;
 
-  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items;
-       it += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t q = it / ng, g = it - q * ng;
+  for (int64_t it = first; it < items; it += step) {
+    const int64_t q = q_next, g = g_next;
+    g_next += step_r;
+    q_next += step_q;
+    if (g_next >= ng) g_next -= ng, ++q_next;
     const int64_t c0 = g * 4, t0 = q * 64;
     const int nb = static_cast<int>((S - 4 * q) < 4 ? (S - 4 * q) : 4);
     uint32_t sfw[4] = {0u, 0u, 0u, 0u};
@@ -180,7 +205,7 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
         float m = 0.0f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[c][i]));
-        const BlockScale bs = block_scale(m, s_enc);
+        const BlockScale bs = block_scale_t(m, s_enc, r_tbl);
         r[c] = bs.r;
         sfw[c] |= bs.sf << (8 * tb);
       }
@@ -232,12 +257,15 @@ __global__ void __launch_bounds__(128) quant_2d_kernel(const uint16_t* __restric
                                                          uint8_t* __restrict__ col_data, uint8_t* __restrict__ col_sf,
                                                          int64_t col_sp, float* __restrict__ col_gs) {
   __shared__ uint32_t tsf[4][32];
+  __shared__ float r_tbl[kRTableSize];
   const float amax = __ldg(amax_dev);
   const float s_enc = encode_scale(amax);
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     if (row_gs) *row_gs = decode_scale(amax);
     if (col_gs) *col_gs = decode_scale(amax);
   }
+  fill_r_table(r_tbl, s_enc);
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t TN = N >> 4, TK = K >> 4;
   const int64_t ctas_k = (TK + 31) >> 5, ctas_n = (TN + 3) >> 2;
@@ -256,7 +284,7 @@ __global__ void __launch_bounds__(128) quant_2d_kernel(const uint16_t* __restric
         mb = max(mb, max(absmax_bits8(__ldg(src)), absmax_bits8(__ldg(src + 1))));
       }
     }
-    const BlockScale bs = block_scale(bf16_bits_to_f32(mb), s_enc);
+    const BlockScale bs = block_scale_t(bf16_bits_to_f32(mb), s_enc, r_tbl);
     tsf[warp][lane] = ok ? bs.sf : 0u;
     if (ok) {
       uint32_t colw[16][2];
@@ -322,6 +350,39 @@ __global__ void sf_pad_zero_kernel(uint8_t* __restrict__ sf, int64_t R, int64_t 
     const int64_t r = e / Sp, c = e - r * Sp;
     if (r >= R || c >= S) sf[sf_offset(r, c, Sp)] = 0;
   }
+}
+
+// ---------------------------------------------------------------------------
+// Self-test of div6_rn against the IEEE division on every non-negative finite
+// float (bit patterns 0 .. 0x7F7FFFFF): counts quotients that differ where the
+// IEEE quotient is a normal float, and E4M3 scale codes that differ anywhere.
+// ---------------------------------------------------------------------------
+__device__ unsigned long long g_div6_bad[2];
+
+__global__ void div6_selftest_kernel() {
+  unsigned long long bad_q = 0, bad_code = 0;
+  for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < 0x7F800000ull;
+       i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+    const float x = __uint_as_float(static_cast<uint32_t>(i));
+    const float a = div6_rn(x), b = __fdiv_rn(x, 6.0f);
+    if (__float_as_uint(a) != __float_as_uint(b) && b >= 1.17549435e-38f) ++bad_q;
+    if (f32_to_e4m3(a) != f32_to_e4m3(b)) ++bad_code;
+  }
+  if (bad_q) atomicAdd(&g_div6_bad[0], bad_q);
+  if (bad_code) atomicAdd(&g_div6_bad[1], bad_code);
+}
+
+cudaError_t selftest_div6(unsigned long long* bad_quotients, unsigned long long* bad_codes, int num_sms) {
+  const unsigned long long zero[2] = {0ull, 0ull};
+  cudaError_t e = cudaMemcpyToSymbol(g_div6_bad, zero, sizeof(zero));
+  if (e != cudaSuccess) return e;
+  div6_selftest_kernel<<<num_sms * 8, 256>>>();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  unsigned long long out[2];
+  if ((e = cudaMemcpyFromSymbol(out, g_div6_bad, sizeof(out))) != cudaSuccess) return e;
+  *bad_quotients = out[0];
+  *bad_codes = out[1];
+  return cudaSuccess;
 }
 
 cudaError_t launch_sf_pad_zero(void* scales, int64_t R, int64_t S, cudaStream_t s) {

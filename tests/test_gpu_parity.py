@@ -340,6 +340,13 @@ def test_linear_fwd_bwd_vs_oracle():
 
 
 # ------------------------------------------------------------------ bounded waits
+def test_block_scale_division_matches_ieee_on_every_float():
+    # the kernels divide by 6 with a corrected reciprocal product; every
+    # non-negative float gives the IEEE quotient where it is normal, and the
+    # same E4M3 scale code everywhere
+    assert api.selftest_scale_division() == (0, 0)
+
+
 def test_wait_probe_times_out_and_reports():
     api.read_device_error(clear=True)
     api.wait_probe(20000)                      # 20 ms; nothing ever arrives
