@@ -6,7 +6,8 @@ its Python binding) never imports it, and it never imports the product.
 
 The arithmetic lives in ``nvfp4_oracle.c`` (plain C, FP32 steps in source order,
 FP64 GEMM); this module only marshals numpy arrays through ctypes.  The readings
-R1..R18 that fix what the pages leave open are listed at the top of that file.
+R1..R18 (NVFP4) and R21..R24 (the MXFP4 comparison format) that fix what the
+pages leave open are listed at the top of that file.
 
 Parity unpinned: the storage layouts (R17 nibble order, R18 scale swizzle) and
 the op-order readings (R4, R6, R9, R16) have no pin in the pages; everything
@@ -60,6 +61,10 @@ def lib():
             "orc_gemm": (None, [_u8p, _u8p, ctypes.c_float, _u8p, _u8p, ctypes.c_float, _i64, _i64,
                                 _i64, _i64p, _i64, _f64p, _f64p]),
             "orc_dequantize": (None, [_u8p, _u8p, ctypes.c_float, _i64, _i64, _f64p]),
+            "orc_e8m0_decode": (ctypes.c_double, [ctypes.c_int]),
+            "orc_mx_scale_exponent": (ctypes.c_int, [ctypes.c_float]),
+            "orc_mx_quantize_row": (None, [_u16p, _i64, _i64, _i64, _u8p, _u8p]),
+            "orc_mx_gemm": (None, [_u8p, _u8p, _u8p, _u8p, _i64, _i64, _i64, _i64p, _i64, _f64p, _f64p]),
             "orc_num_threads": (ctypes.c_int, []),
         }
         for name, (res, args) in sig.items():
@@ -246,6 +251,49 @@ def dequantize(codes, sf, sg):
     out = np.zeros((R, C), dtype=np.float64)
     lib().orc_dequantize(_p(codes, _u8p), _p(sf, _u8p), float(sg), R, C, _p(out, _f64p))
     return out
+
+
+# ---------------------------------------------------------------- MXFP4 (R21-R24)
+def e8m0_decode(byte):
+    return lib().orc_e8m0_decode(int(byte))
+
+
+def mx_scale_exponent(bamax):
+    return lib().orc_mx_scale_exponent(float(bamax))
+
+
+def mx_quantize_row(x):
+    """Row-wise 1x32 MXFP4.  Returns (codes [R, C] u8, sf [R, C/32] UE8M0 bytes)."""
+    x = _bf16_bits(x)
+    R, C = x.shape
+    codes = np.zeros((R, C), dtype=np.uint8)
+    sf = np.zeros((R, C // 32), dtype=np.uint8)
+    lib().orc_mx_quantize_row(_p(x, _u16p), R, C, C, _p(codes, _u8p), _p(sf, _u8p))
+    return codes, sf
+
+
+def mx_dequantize(codes, sf):
+    """FP64 values of an unpacked MXFP4 operand (codes [R, C], sf [R, C/32])."""
+    grid = np.array([lib().orc_e2m1_decode(c) for c in range(16)])
+    scale = np.array([lib().orc_e8m0_decode(b) for b in range(256)])
+    return grid[codes] * np.repeat(scale[sf], 32, axis=1)
+
+
+def mx_gemm(ca, sa, cb, sb, pairs=None):
+    """FP64 D = dq(A) dq(B)^T on MXFP4 operands.  Full [M, N] or sampled entries.  Returns (D, absum)."""
+    ca, sa, cb, sb = (np.ascontiguousarray(t, dtype=np.uint8) for t in (ca, sa, cb, sb))
+    M, K = ca.shape
+    N = cb.shape[0]
+    assert cb.shape[1] == K and sa.shape == (M, K // 32) and sb.shape == (N, K // 32)
+    pr = None if pairs is None else np.ascontiguousarray(pairs, dtype=np.int64)
+    n = M * N if pr is None else pr.shape[0]
+    D = np.zeros(n, dtype=np.float64)
+    S = np.zeros(n, dtype=np.float64)
+    lib().orc_mx_gemm(_p(ca, _u8p), _p(sa, _u8p), _p(cb, _u8p), _p(sb, _u8p), M, N, K,
+                      None if pr is None else _p(pr, _i64p), 0 if pr is None else n, _p(D, _f64p), _p(S, _f64p))
+    if pr is None:
+        D, S = D.reshape(M, N), S.reshape(M, N)
+    return D, S
 
 
 def num_threads():

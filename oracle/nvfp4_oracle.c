@@ -41,6 +41,18 @@
  *   R16 RHT FP32 order: signs, butterflies h = 1,2,4,8, then * 0.25
  *   R17 packing: element 2i in the low nibble, 2i+1 in the high nibble
  *   R18 scale layout: 128x4 tiles of 512 bytes (see orc_sf_offset)
+ * MXFP4, the format the pages compare NVFP4 against ("Pretraining Large Language
+ * Models with NVFP4", section 2A: blocks of 32 instead of 16, UE8M0 instead of
+ * E4M3 block scales; section 3: the 8B comparison), read as the OCP
+ * Microscaling v1.0 format the name refers to:
+ *   R21 1x32 blocks along K, one UE8M0 scale each, no per-tensor scale
+ *   R22 UE8M0 byte e decodes to 2^(e-127); 0xFF (NaN) is never produced
+ *   R23 scale 2^s with s = floor(log2(bamax)) - 2 (2 = exponent of E2M1's
+ *       largest power of two: 6 = 1.5 * 2^2), clamped to [-127, 127]; an
+ *       all-zero block gets s = -127 (byte 0)
+ *   R24 elements: y = x * 2^-s (exact), then E2M1 round-to-nearest-even with
+ *       saturation at 6 (R1, R2) -- so a block whose max is in [6*2^s, 8*2^s)
+ *       clips its largest values to 6 * 2^s
  * Floating point: built with -ffp-contract=off and without fast-math, so every
  * FP32 operation below is one IEEE operation in the order written.
  */
@@ -432,6 +444,76 @@ void orc_dequantize(const uint8_t *codes, const uint8_t *sf, float sg, int64_t R
     for (int64_t r = 0; r < R; r++)
         for (int64_t c = 0; c < C; c++)
             out[r * C + c] = orc_e2m1_decode(codes[r * C + c]) * orc_e4m3_decode(sf[r * S + c / 16]) * (double)sg;
+}
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4 (R21-R24): the comparison format of section 2A / section 3.         */
+/* ------------------------------------------------------------------------ */
+double orc_e8m0_decode(int byte)                        /* R22 */
+{
+    if ((byte & 0xFF) == 0xFF) return NAN;
+    return ldexp(1.0, (byte & 0xFF) - 127);
+}
+
+/* s = floor(log2(bamax)) - 2, clamped to [-127, 127] (R23).  frexp writes
+ * bamax = m * 2^e with m in [0.5, 1), so floor(log2(bamax)) = e - 1 exactly,
+ * subnormal inputs included. */
+int orc_mx_scale_exponent(float bamax)
+{
+    if (bamax == 0.0f) return -127;
+    int e;
+    frexp((double)bamax, &e);
+    int s = (e - 1) - 2;
+    if (s < -127) s = -127;
+    if (s > 127) s = 127;
+    return s;
+}
+
+/* Row-wise 1x32 MXFP4 quantization (R21-R24): codes [R, C] one code per byte,
+ * sf [R, C/32] UE8M0 bytes. */
+void orc_mx_quantize_row(const uint16_t *x, int64_t R, int64_t C, int64_t ld, uint8_t *codes, uint8_t *sf)
+{
+    int64_t S = C / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t b = 0; b < S; b++) {
+            float v[32], bamax = 0.0f;
+            for (int i = 0; i < 32; i++) {
+                v[i] = bf16_to_f32(x[r * ld + b * 32 + i]);
+                float a = fabsf(v[i]);
+                if (a > bamax) bamax = a;
+            }
+            int s_exp = orc_mx_scale_exponent(bamax);
+            sf[r * S + b] = (uint8_t)(s_exp + 127);
+            for (int i = 0; i < 32; i++) {
+                float y = (float)ldexp((double)v[i], -s_exp);   /* exact: a power-of-two scale (R24) */
+                codes[r * C + b * 32 + i] = (uint8_t)orc_e2m1_encode_rn(y);
+            }
+        }
+}
+
+/* GEMM on MXFP4 operands: codes [rows, K], UE8M0 scales [rows, K/32]; same
+ * output convention as orc_gemm. */
+void orc_mx_gemm(const uint8_t *ca, const uint8_t *sa, const uint8_t *cb, const uint8_t *sb,
+                 int64_t M, int64_t N, int64_t K, const int64_t *pairs, int64_t npairs, double *D,
+                 double *absum)
+{
+    int64_t S = K / 32;
+    int64_t total = pairs ? npairs : M * N;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t t = 0; t < total; t++) {
+        int64_t m = pairs ? pairs[2 * t] : t / N;
+        int64_t n = pairs ? pairs[2 * t + 1] : t % N;
+        double acc = 0.0, aacc = 0.0;
+        for (int64_t k = 0; k < K; k++) {
+            double a = orc_e2m1_decode(ca[m * K + k]) * orc_e8m0_decode(sa[m * S + k / 32]);
+            double b = orc_e2m1_decode(cb[n * K + k]) * orc_e8m0_decode(sb[n * S + k / 32]);
+            acc += a * b;
+            aacc += fabs(a * b);
+        }
+        D[t] = acc;
+        absum[t] = aacc;
+    }
 }
 
 int orc_num_threads(void)
