@@ -139,6 +139,31 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, n
                         int64_t ldd, nvfp4_stream_t stream);
 
 /*
+ * MXFP4, the format the NVFP4 page compares against ("Pretraining Large
+ * Language Models with NVFP4", section 2A: blocks of 32 elements with UE8M0
+ * scales instead of 16 with E4M3 scales; section 3: the 8B-model comparison).
+ * Read as the OCP Microscaling format: one UE8M0 byte e (value 2^(e-127)) per
+ * 1x32 block along K, no per-tensor scale.  An MXFP4 operand is an
+ * nvfp4_tensor whose scales are UE8M0 bytes of blocks of 32, in the same
+ * 128x4 tile layout with Sp = pad4(cols/32); its global_scale holds 1.0.
+ *
+ * nvfp4_mx_scale_bytes: bytes of the UE8M0 scales of a [rows, cols] operand.
+ * nvfp4_mx_quantize: BF16 x [R, C] (pitch ld) -> out (rows R, cols C), row-wise
+ *   1x32 blocks, C % 32 == 0: scale 2^s with s = floor(log2 max|block|) - 2
+ *   clamped to [-127, 127] (all-zero block: s = -127); codes = E2M1
+ *   round-to-nearest-even of x * 2^-s, saturating at 6.  Writes 1.0 to
+ *   out->global_scale.
+ * nvfp4_mx_gemm: D = sum_k dq(A[m, k]) dq(B[n, k]) on MXFP4 operands, FP32
+ *   accumulation, D as in nvfp4_gemm.  Needs K % 64 == 0 and M, N multiples
+ *   of 256 (it runs on the CTA-pair kernel; other shapes: NVFP4_ERR_SHAPE).
+ */
+size_t nvfp4_mx_scale_bytes(int64_t rows, int64_t cols);
+nvfp4_status nvfp4_mx_quantize(const void* x, int64_t R, int64_t C, int64_t ld, const nvfp4_tensor* out,
+                               nvfp4_stream_t stream);
+nvfp4_status nvfp4_mx_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, nvfp4_out_dtype out_dtype,
+                           int64_t ldd, nvfp4_stream_t stream);
+
+/*
  * Linear layer Y = X W^T with X [T, Cin], W [Cout, Cin] (BF16, contiguous).
  * Workspace (device, caller-owned, nvfp4_linear_workspace_bytes bytes) holds
  * the quantized operands; linear_fwd leaves in it what linear_bwd needs.

@@ -54,6 +54,9 @@ PROTOTYPES = {
     "nvfp4_status_string": (_c.c_char_p, [_int]),
     "nvfp4_version": (_int, []),
     "nvfp4_last_cuda_error": (_int, [_c.POINTER(_c.c_char_p)]),
+    "nvfp4_mx_scale_bytes": (_c.c_size_t, [_i64, _i64]),
+    "nvfp4_mx_quantize": (_int, [_vp, _i64, _i64, _i64, _tp, _vp]),
+    "nvfp4_mx_gemm": (_int, [_tp, _tp, _vp, _int, _i64, _vp]),
     "nvfp4_selftest_scale_division": (_int, [_c.POINTER(_c.c_uint64), _c.POINTER(_c.c_uint64)]),
 }
 

@@ -97,6 +97,36 @@ def gemm(A, B, out_dtype=OUT_F32, out=None):
     return out
 
 
+# ---------------------------------------------------------------- MXFP4 comparison format
+def mx_scale_bytes(rows, cols):
+    return lib().nvfp4_mx_scale_bytes(rows, cols)
+
+
+def mx_quantize(x, out=None):
+    """BF16 [R, C] -> MXFP4 QTensor (1x32 blocks along C, UE8M0 scales, global_scale = 1)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    R, C = x.shape
+    if out is None:
+        out = QTensor(torch.empty(R, C // 2, dtype=torch.uint8, device=x.device),
+                      torch.empty(mx_scale_bytes(R, C), dtype=torch.uint8, device=x.device),
+                      torch.empty(1, dtype=torch.float32, device=x.device), R, C)
+    d = out.desc()
+    check("nvfp4_mx_quantize", lib().nvfp4_mx_quantize(x.data_ptr(), R, C, x.stride(0), ctypes.byref(d),
+                                                       _stream(x.device)))
+    return out
+
+
+def mx_gemm(A, B, out_dtype=OUT_F32, out=None):
+    """D[M, N] = sum_k A[m, k] B[n, k] on MXFP4 operands (FP32 accumulation)."""
+    dt = torch.float32 if out_dtype == OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty(A.rows, B.rows, dtype=dt, device=A.data.device)
+    ad, bd = A.desc(), B.desc()
+    check("nvfp4_mx_gemm", lib().nvfp4_mx_gemm(ctypes.byref(ad), ctypes.byref(bd), out.data_ptr(), out_dtype,
+                                               out.stride(0), _stream(out.device)))
+    return out
+
+
 class LinearWorkspace:
     """Caller-owned workspace of the linear layer (quantized operands + scalars)."""
 

@@ -124,6 +124,41 @@ size_t nvfp4_scale_bytes(int64_t rows, int64_t cols) {
   return (rows > 0 && cols > 0) ? static_cast<size_t>(pad128(rows) * pad4(cols / 16)) : 0;
 }
 
+size_t nvfp4_mx_scale_bytes(int64_t rows, int64_t cols) {
+  return (rows > 0 && cols > 0) ? static_cast<size_t>(pad128(rows) * pad4(cols / 32)) : 0;
+}
+
+nvfp4_status nvfp4_mx_quantize(const void* x, int64_t R, int64_t C, int64_t ld, const nvfp4_tensor* out,
+                               nvfp4_stream_t stream) {
+  if (!x || !out) return NVFP4_ERR_INVALID_ARG;
+  if (R <= 0 || C <= 0 || ld < C || C % 32) return NVFP4_ERR_SHAPE;
+  if (!aligned16(x) || ld % 8) return NVFP4_ERR_ALIGN;
+  nvfp4_status st;
+  if ((st = check_tensor(out, R, C)) != NVFP4_OK) return st;
+  DeviceInfo di;
+  if ((st = device_info(&di)) != NVFP4_OK) return st;
+  return cuda_status(nvfp4::launch_mx_quant_row(x, R, C, ld, out->data, out->scales, out->global_scale, di.sms,
+                                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_mx_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, nvfp4_out_dtype out_dtype,
+                           int64_t ldd, nvfp4_stream_t stream) {
+  if (!A || !B || !D) return NVFP4_ERR_INVALID_ARG;
+  if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
+  const int64_t M = A->rows, N = B->rows, K = A->cols;
+  if (M <= 0 || N <= 0 || K <= 0 || B->cols != K) return NVFP4_ERR_SHAPE;
+  if (K % 64 || M % 256 || N % 256 || ldd < N || M >= (1LL << 31) || N >= (1LL << 31) || K >= (1LL << 31))
+    return NVFP4_ERR_SHAPE;
+  nvfp4_status st;
+  if ((st = check_tensor(A, M, K)) != NVFP4_OK || (st = check_tensor(B, N, K)) != NVFP4_OK) return st;
+  if (!aligned16(D) || ldd % 8) return NVFP4_ERR_ALIGN;
+  DeviceInfo di;
+  if ((st = device_info(&di)) != NVFP4_OK) return st;
+  return cuda_status(nvfp4::launch_gemm(A->data, A->scales, A->global_scale, B->data, B->scales, B->global_scale,
+                                        M, N, K, D, out_dtype == NVFP4_OUT_BF16, ldd, di.sms,
+                                        reinterpret_cast<cudaStream_t>(stream), 1));
+}
+
 uint32_t nvfp4_rht_sign_mask(void) { return sign_mask(); }
 
 nvfp4_status nvfp4_selftest_scale_division(uint64_t* bad_quotients, uint64_t* bad_codes) {

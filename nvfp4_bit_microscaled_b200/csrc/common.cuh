@@ -468,6 +468,22 @@ __device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, u
       : "memory");
 }
 
+// MXFP4 form: E2M1 operands with one UE8M0 scale per 32 elements (two per
+// K=64 step).  A 32-bit tensor-memory scale cell holds the four scales of two
+// consecutive K steps; the byte pair a step uses is named by the scale-factor
+// id in the instruction descriptor (bits 29-30 for A, 4-5 for B) and by bits
+// 30-31 of the scale address, 0 for the first step and 2 for the second.
+__device__ __forceinline__ void mma_mxf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t"
+      "}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive, in every CTA of cta_mask, on the mbarrier at this shared-memory
 // offset once the pair MMAs issued so far by this thread have completed.
 __device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t cta_mask) {

@@ -352,13 +352,35 @@ static_assert(P_OFF_STG % 1024 == 0, "swizzled staging boxes need 1024-byte alig
 static_assert(P_SMEM_BYTES <= 232448, "pair kernel shared memory exceeds the per-block limit");
 constexpr int P_GROUP_M = 8;
 
-// kind::mxf4nvf4, A/B E2M1 K-major, UE4M3 scales, M = 256 (pair), N = 256.
-__host__ __device__ constexpr uint32_t make_idesc_pair() {
-  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(256 >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
+// kind::mxf4nvf4 (NVFP4: UE4M3 scales) or kind::mxf4 (MXFP4: UE8M0 scales,
+// bit 23), A/B E2M1 K-major, M = 256 (pair), N = 256.
+__host__ __device__ constexpr uint32_t make_idesc_pair(bool mx) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(256 >> 3) << 17) | (mx ? (1u << 23) : 0u) |
+         (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
+// One K = 64 MMA step kb (0..3) of a stage.  NVFP4: scale tile kb, all four
+// bytes of its cells.  MXFP4: scale tile kb/2, byte pair 2*(kb%2).
+template <bool MX>
+__device__ __forceinline__ void pair_mma_step(uint32_t acc, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t sfa_t, uint32_t sfb_t, int kb, bool accumulate) {
+  if (MX) {
+    const uint32_t sid = 2u * static_cast<uint32_t>(kb & 1);
+    const int atom = kb >> 1;
+    mma_mxf4_pair(acc, adesc + 2 * kb, bdesc + 2 * kb, idesc | (sid << 29) | (sid << 4),
+                  (sfa_t + 4 * atom) | (sid << 30), (sfb_t + 8 * atom) | (sid << 30), accumulate);
+  } else {
+    mma_nvf4_pair(acc, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa_t + 4 * kb, sfb_t + 8 * kb, accumulate);
+  }
+}
+
+// MX selects the MXFP4 operand format: one UE8M0 scale per 32 elements, so a
+// 128x4 scale tile covers K = 128 (two MMA steps) instead of K = 64, a stage
+// carries two scale tiles per 128 rows instead of four, and each MMA step
+// names its byte pair of the scale cell (see mma_mxf4_pair).
+template <bool MX>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmD, const uint8_t* __restrict__ sfa,
                       const uint8_t* __restrict__ sfb, const float* __restrict__ gsa,
                       const float* __restrict__ gsb, int M, int N, int K, int out_bf16) {
@@ -379,7 +401,9 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
   const int num_m = M / 256, num_n = N / 256;
   const int num_tiles = num_m * num_n;
-  const int katoms = (K + 63) / 64;
+  const int katoms = (K + 63) / 64;                     // MMA steps of K = 64
+  const int sf_atoms = MX ? (K + 127) / 128 : katoms;   // 128x4 scale tiles along K
+  constexpr int ATOMS_PER_STAGE = MX ? KB_PER_STAGE / 2 : KB_PER_STAGE;
   const int num_kt = (K + 255) / 256;
 
   if (threadIdx.x == 0) {
@@ -422,7 +446,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
       for (int kt = 0; kt < num_kt; ++kt) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, kErrWaitEmpty)) { *abort_flag = 1; break; }
         const int nkb = min(KB_PER_STAGE, katoms - kt * KB_PER_STAGE);
-        const uint32_t sf_bytes = static_cast<uint32_t>(nkb) * 512u;
+        const uint32_t sf_bytes = static_cast<uint32_t>(MX ? (nkb + 1) / 2 : nkb) * 512u;
         if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (P_A_BYTES + P_B_BYTES));
         tma_load_2d_pair(smem + P_OFF_A + stage * P_A_BYTES, &tmA, full_l + stage * 8, kt * BK_BYTES,
                          tm * 256 + 128 * static_cast<int>(rank));
@@ -430,11 +454,11 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                          tn * 256 + 128 * static_cast<int>(rank));
         mbar_arrive_expect_tx(&sfd_full[stage], 3 * sf_bytes);
         bulk_load(smem + P_OFF_SFA + stage * P_SFA_BYTES,
-                  sfa + (static_cast<int64_t>(2 * tm + rank) * katoms + kt * KB_PER_STAGE) * 512, sf_bytes,
+                  sfa + (static_cast<int64_t>(2 * tm + rank) * sf_atoms + kt * ATOMS_PER_STAGE) * 512, sf_bytes,
                   &sfd_full[stage]);
         for (int h = 0; h < 2; ++h)
           bulk_load(smem + P_OFF_SFB + stage * P_SFB_BYTES + h * KB_PER_STAGE * 512,
-                    sfb + (static_cast<int64_t>(2 * tn + h) * katoms + kt * KB_PER_STAGE) * 512, sf_bytes,
+                    sfb + (static_cast<int64_t>(2 * tn + h) * sf_atoms + kt * ATOMS_PER_STAGE) * 512, sf_bytes,
                     &sfd_full[stage]);
         issued[stage] = true;
         issued_parity[stage] = phase;
@@ -452,7 +476,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     int stage = 0;
     uint32_t phase = 0, acc_phase = 0;
     const uint32_t a_base = smem_u32(smem + P_OFF_A), b_base = smem_u32(smem + P_OFF_B);
-    const uint32_t idesc = make_idesc_pair();
+    const uint32_t idesc = make_idesc_pair(MX);
     // Stage descriptors differ only in the start-address field (address >> 4,
     // bits 0-13): adding stage * bytes / 16 moves to the stage's tile.
     const uint64_t adesc0 = smem_desc(a_base, 16, 1024, 2), bdesc0 = smem_desc(b_base, 16, 1024, 2);
@@ -474,14 +498,11 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         if ((kt + 1) * KB_PER_STAGE <= katoms) {
           // full stage: four MMAs back to back, nothing else between them
 #pragma unroll
-          for (int kb = 0; kb < KB_PER_STAGE; ++kb)
-            mma_nvf4_pair(tmem + ACC_COL, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa_t + 4 * kb, sfb_t + 8 * kb,
-                          (kt | kb) != 0);
+          for (int kb = 0; kb < KB_PER_STAGE; ++kb) pair_mma_step<MX>(tmem + ACC_COL, adesc, bdesc, idesc, sfa_t, sfb_t, kb, (kt | kb) != 0);
         } else {
           const int nkb = katoms - kt * KB_PER_STAGE;
           for (int kb = 0; kb < nkb; ++kb)
-            mma_nvf4_pair(tmem + ACC_COL, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa_t + 4 * kb, sfb_t + 8 * kb,
-                          (kt | kb) != 0);
+            pair_mma_step<MX>(tmem + ACC_COL, adesc, bdesc, idesc, sfa_t, sfb_t, kb, (kt | kb) != 0);
         }
         tc_commit_pair_mc(&empty[stage], 0x3);
         if (++stage == P_STAGES) stage = 0, phase ^= 1u;
@@ -506,15 +527,16 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
           break;
         }
         const int nkb = min(KB_PER_STAGE, katoms - kt * KB_PER_STAGE);
+        const int natoms = MX ? (nkb + 1) / 2 : nkb;   // scale tiles this stage carries
         const uint8_t* sa = smem + P_OFF_SFA + stage * P_SFA_BYTES + lane * 16;
         const uint8_t* sb = smem + P_OFF_SFB + stage * P_SFB_BYTES + lane * 16;
         uint32_t ra[16], rb[32];
 #pragma unroll
         for (int kb = 0; kb < KB_PER_STAGE; ++kb) {
-          const uint4 va = kb < nkb ? *reinterpret_cast<const uint4*>(sa + 512 * kb) : make_uint4(0, 0, 0, 0);
-          const uint4 v0 = kb < nkb ? *reinterpret_cast<const uint4*>(sb + 512 * kb) : make_uint4(0, 0, 0, 0);
-          const uint4 v1 =
-              kb < nkb ? *reinterpret_cast<const uint4*>(sb + KB_PER_STAGE * 512 + 512 * kb) : make_uint4(0, 0, 0, 0);
+          const uint4 va = kb < natoms ? *reinterpret_cast<const uint4*>(sa + 512 * kb) : make_uint4(0, 0, 0, 0);
+          const uint4 v0 = kb < natoms ? *reinterpret_cast<const uint4*>(sb + 512 * kb) : make_uint4(0, 0, 0, 0);
+          const uint4 v1 = kb < natoms ? *reinterpret_cast<const uint4*>(sb + KB_PER_STAGE * 512 + 512 * kb)
+                                       : make_uint4(0, 0, 0, 0);
           ra[4 * kb + 0] = va.x; ra[4 * kb + 1] = va.y; ra[4 * kb + 2] = va.z; ra[4 * kb + 3] = va.w;
           rb[8 * kb + 0] = v0.x; rb[8 * kb + 1] = v0.y; rb[8 * kb + 2] = v0.z; rb[8 * kb + 3] = v0.w;
           rb[8 * kb + 4] = v1.x; rb[8 * kb + 5] = v1.y; rb[8 * kb + 6] = v1.z; rb[8 * kb + 7] = v1.w;
@@ -674,7 +696,7 @@ bool make_output_map(CUtensorMap* tm, void* D, int64_t M, int64_t N, int64_t ldd
 
 cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a_gs, const void* b_data,
                         const void* b_scales, const float* b_gs, int64_t M, int64_t N, int64_t K, void* D,
-                        int out_bf16, int64_t ldd, int num_sms, cudaStream_t s) {
+                        int out_bf16, int64_t ldd, int num_sms, cudaStream_t s, int mx) {
   // The pair kernel stores through TMA: the output base must be 16-byte
   // aligned and its row stride a multiple of 16 bytes.
   const int64_t esize = out_bf16 ? 2 : 4;
@@ -684,12 +706,14 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
   if (!make_operand_map(&tmA, a_data, M, K, BM) || !make_operand_map(&tmB, b_data, N, K, pair ? 128 : BN))
     return cudaErrorInvalidValue;
   if (pair && !make_output_map(&tmD, D, M, N, ldd, out_bf16)) return cudaErrorInvalidValue;
+  if (mx && !pair) return cudaErrorInvalidValue;  // MXFP4 runs on the CTA-pair kernel only
   const auto* sa = static_cast<const uint8_t*>(a_scales);
   const auto* sb = static_cast<const uint8_t*>(b_scales);
   if (pair) {
-    static int max_pairs = -1;
-    if (max_pairs < 0) {
-      cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    static int max_pairs[2] = {-1, -1};
+    auto kern = mx ? gemm_fp4_pair_kernel<true> : gemm_fp4_pair_kernel<false>;
+    if (max_pairs[mx ? 1 : 0] < 0) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(P_SMEM_BYTES));
       if (e != cudaSuccess) return e;
       cudaLaunchConfig_t q = {};
@@ -704,12 +728,13 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
       q.attrs = qa;
       q.numAttrs = 1;
       int n = 0;
-      e = cudaOccupancyMaxActiveClusters(&n, gemm_nvf4_pair_kernel, &q);
+      e = cudaOccupancyMaxActiveClusters(&n, kern, &q);
       if (e != cudaSuccess || n < 1) n = num_sms / 2;
-      max_pairs = n;
+      max_pairs[mx ? 1 : 0] = n;
     }
     const int64_t tiles = (M / 256) * (N / 256);
-    const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+    const int mp = max_pairs[mx ? 1 : 0];
+    const int pairs = static_cast<int>(tiles < mp ? tiles : mp);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
     cfg.blockDim = dim3(NUM_THREADS);
@@ -722,7 +747,7 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel, tmA, tmB, tmD, sa, sb, a_gs, b_gs, static_cast<int>(M),
+    return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmD, sa, sb, a_gs, b_gs, static_cast<int>(M),
                               static_cast<int>(N), static_cast<int>(K), out_bf16);
   }
   static bool attr_set = false;

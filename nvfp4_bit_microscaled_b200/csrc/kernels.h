@@ -20,6 +20,11 @@ cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, co
                              uint32_t sign_mask, int sr, uint64_t seed, void* data, void* scales,
                              float* gs_out, int num_sms, cudaStream_t s);
 
+// MXFP4 row-wise 1x32 quantization: data [R, C/2], UE8M0 scales in the 128x4
+// tile layout with sp = pad4(C/32); writes 1.0 to *gs_out when given.
+cudaError_t launch_mx_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, void* data, void* scales,
+                                float* gs_out, int num_sms, cudaStream_t s);
+
 // 2D 16x16 quantization of W [N, K]: row copy [N, K/2] and/or column copy [K, N/2].
 cudaError_t launch_quant_2d(const void* w, int64_t N, int64_t K, int64_t ld, const float* amax_dev,
                             void* row_data, void* row_scales, float* row_gs, void* col_data, void* col_scales,
@@ -32,10 +37,12 @@ cudaError_t selftest_div6(unsigned long long* bad_quotients, unsigned long long*
 // Zero the padding of a scale matrix (rows >= R or scale columns >= S).
 cudaError_t launch_sf_pad_zero(void* scales, int64_t R, int64_t S, cudaStream_t s);
 
-// Block-scaled FP4 GEMM: D[M,N] = sgA * sgB * sum_k A[m,k] B[n,k].
+// Block-scaled FP4 GEMM: D[M,N] = sgA * sgB * sum_k A[m,k] B[n,k].  mx != 0:
+// MXFP4 operands (UE8M0 scale per 32 elements, sgA = sgB = 1 pointers still
+// read), M and N multiples of 256 only.
 cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a_gs, const void* b_data,
                         const void* b_scales, const float* b_gs, int64_t M, int64_t N, int64_t K, void* D,
-                        int out_bf16, int64_t ldd, int num_sms, cudaStream_t s);
+                        int out_bf16, int64_t ldd, int num_sms, cudaStream_t s, int mx = 0);
 
 // Bounded-wait self-test: a kernel waits on an mbarrier nobody arrives on.
 cudaError_t launch_wait_probe(uint32_t timeout_us, cudaStream_t s);

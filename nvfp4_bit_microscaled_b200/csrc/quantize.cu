@@ -342,6 +342,67 @@ __global__ void __launch_bounds__(128) quant_2d_kernel(const uint16_t* __restric
 }
 
 // ---------------------------------------------------------------------------
+// MXFP4 row-wise 1x32 (the comparison format of "Pretraining Large Language
+// Models with NVFP4", section 2A: 32-element blocks, UE8M0 scales, no tensor
+// scale), OCP Microscaling rule: scale 2^s with s = floor(log2 bamax) - 2,
+// clamped to [-127, 127]; codes = E2M1 round-to-nearest-even of x * 2^-s,
+// saturating at 6.  For a BF16 block maximum with exponent field e (bias 127,
+// e = 0 for zero and subnormals) that is the UE8M0 byte max(e, 2) - 2, and
+// 2^-s is the float with exponent field 254 - byte, so every step is exact.
+// Warp item: one row segment of 32 blocks (1024 elements); lane = one block
+// (four 16-byte loads, one 16-byte store); the four scale bytes of a scale
+// word meet by shuffle.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256, 4) mx_quant_row_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+                                                             int64_t ld, uint8_t* __restrict__ data,
+                                                             uint8_t* __restrict__ sf, int64_t sp,
+                                                             float* __restrict__ gs_out) {
+  if (blockIdx.x == 0 && threadIdx.x == 0 && gs_out) *gs_out = 1.0f;  // no tensor-level scale
+  const int lane = threadIdx.x & 31;
+  const int64_t S = C >> 5;
+  const int64_t nseg = (S + 31) >> 5;
+  const int64_t items = R * nseg;
+  const int64_t half_c = C >> 1;
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t step = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5), step_q = step / nseg,
+                step_r = step - step_q * nseg;
+  int64_t row = first / nseg, seg = first - row * nseg;
+  for (int64_t it = first; it < items; it += step) {
+    const int64_t r = row, b = seg * 32 + lane;
+    seg += step_r;
+    row += step_q;
+    if (seg >= nseg) seg -= nseg, ++row;
+    const bool ok = b < S;
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = make_uint4(0, 0, 0, 0);
+    if (ok) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + r * ld + b * 32);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = __ldcs(src + j);
+    }
+    const uint32_t mb = max(max(absmax_bits8(v[0]), absmax_bits8(v[1])), max(absmax_bits8(v[2]), absmax_bits8(v[3])));
+    const uint32_t e = mb >> 7;                       // BF16 exponent field of the block maximum
+    const uint32_t byte = e > 2u ? e - 2u : 0u;       // UE8M0 scale byte = s + 127
+    const float p = __uint_as_float((254u - byte) << 23);  // 2^-s
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float y[8];
+      unpack8(v[j], y);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(y[i], p);
+      w[j] = pack8(y);
+    }
+    if (ok) *reinterpret_cast<uint4*>(data + r * half_c + b * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    uint32_t word = ok ? (byte << (8 * (lane & 3))) : 0u;
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+    if ((lane & 3) == 0 && ok) *reinterpret_cast<uint32_t*>(sf + sf_offset(r, b, sp)) = word;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Padding of the scale matrix (rows R..pad128(R), scale columns S..pad4(S)).
 // ---------------------------------------------------------------------------
 __global__ void sf_pad_zero_kernel(uint8_t* __restrict__ sf, int64_t R, int64_t S, int64_t Rp, int64_t Sp) {
@@ -441,6 +502,18 @@ cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, co
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_sf_pad_zero(scales, C, S, s);
+}
+
+cudaError_t launch_mx_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, void* data, void* scales,
+                                float* gs_out, int num_sms, cudaStream_t s) {
+  const int64_t S = C / 32, sp = (S + 3) / 4 * 4;
+  const int64_t warp_items = R * ((S + 31) / 32);
+  const int grid = grid_for(warp_items, 8, num_sms, 8);
+  mx_quant_row_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), R, C, ld, static_cast<uint8_t*>(data),
+                                           static_cast<uint8_t*>(scales), sp, gs_out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_sf_pad_zero(scales, R, S, s);
 }
 
 cudaError_t launch_quant_2d(const void* w, int64_t N, int64_t K, int64_t ld, const float* amax_dev,

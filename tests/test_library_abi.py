@@ -90,3 +90,20 @@ def test_argument_checks_return_before_any_launch(L):
     assert L.nvfp4_linear_fwd(fake, fake, 100, 64, 64, fake, fake, 1 << 30, None) == 2
     assert L.nvfp4_linear_fwd(fake, fake, 64, 64, 64, fake, fake, 16, None) == 7        # workspace too small
     assert L.nvfp4_linear_bwd(fake, 64, 64, 64, 0, fake, fake, None, 1 << 30, None) == 7
+
+
+def test_mx_sizes_and_argument_checks(L):
+    assert L.nvfp4_mx_scale_bytes(128, 256) == 128 * 8
+    assert L.nvfp4_mx_scale_bytes(130, 96) == 256 * 4          # rows pad to 128, scale cols (3) to 4
+    fake = 1 << 20
+    q = L.nvfp4_mx_quantize
+    assert q(fake, 16, 48, 48, ctypes.byref(_t(16, 48)), None) == 2          # C % 32
+    assert q(fake, 16, 64, 64, ctypes.byref(_t(16, 32)), None) == 2          # descriptor shape
+    assert q(fake + 8, 16, 64, 64, ctypes.byref(_t(16, 64)), None) == 3      # misaligned input
+    assert q(fake, 16, 64, 64, None, None) == 1
+    g = L.nvfp4_mx_gemm
+    a, b = _t(256, 256), _t(256, 256)
+    assert g(ctypes.byref(_t(128, 256)), ctypes.byref(b), fake, 0, 256, None) == 2   # M % 256
+    assert g(ctypes.byref(a), ctypes.byref(_t(384, 256)), fake, 0, 384, None) == 2   # N % 256
+    assert g(ctypes.byref(_t(256, 96)), ctypes.byref(_t(256, 96)), fake, 0, 256, None) == 2  # K % 64
+    assert g(ctypes.byref(a), ctypes.byref(b), fake + 4, 0, 256, None) == 3        # misaligned D
