@@ -509,7 +509,44 @@ def run_reference(args, rank, world):
 
 
 CASES = ("gemm", "amax", "amax_rht", "amax_both", "quant_row", "quant_row_sr", "quant_2d", "quant_col_rht",
-         "quant_col_rht_sr")
+         "quant_col_rht_sr", "mx_gemm", "mx_quant_row")
+
+
+def _event_ms(fn, reps):
+    """Average device time of fn() over reps launches on the current stream."""
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(reps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / reps
+
+
+def measure_mxfp4(X, W, reps=20):
+    """The MXFP4 comparison format on the fprop operands of the workload:
+    1x32 UE8M0 quantization of X and W, then Y = X W^T (BF16 out) on the
+    block-32 CTA-pair kernel.  Timed on its own, after the step timing."""
+    T, Ci = X.shape
+    Co = W.shape[0]
+    qx, qw = api.mx_quantize(X), api.mx_quantize(W)
+    Y = torch.empty(T, Co, dtype=torch.bfloat16, device=X.device)
+    for _ in range(3):
+        api.mx_quantize(X, out=qx)
+        api.mx_gemm(qx, qw, api.OUT_BF16, out=Y)
+    torch.cuda.synchronize()
+    q_ms = _event_ms(lambda: api.mx_quantize(X, out=qx), reps)
+    g_ms = _event_ms(lambda: api.mx_gemm(qx, qw, api.OUT_BF16, out=Y), reps)
+    peaks, _ = load_peaks()
+    fp4_peak = FP4_PER_BF16 * peaks["bf16_tflops_sustained"]
+    q_bytes = T * Ci * (2 + 0.5 + 1 / 32)
+    tflops = 2.0 * T * Co * Ci / (g_ms * 1e-3) / 1e12
+    gbs = q_bytes / (q_ms * 1e-3) / 1e9
+    return {"gemm_fprop": {"ms_per_launch": round(g_ms, 4), "tflops": round(tflops, 1),
+                           "frac_fp4_peak": round(tflops / fp4_peak, 4)},
+            "quant_row_x": {"ms_per_launch": round(q_ms, 4), "gbs": round(gbs, 1),
+                            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)},
+            "note": "comparison format (1x32 blocks, UE8M0 scales, no tensor scale); not part of the step"}
 
 
 def run_case(args):
@@ -522,7 +559,19 @@ def run_case(args):
     from nvfp4_bit_microscaled_b200 import build as libbuild
     libbuild.build()
     amax = torch.zeros(1, dtype=torch.float32, device=dev)
-    if args.case == "gemm":
+    if args.case == "mx_gemm":
+        M, N, K = shape
+        qa = api.mx_quantize(synth.activations(M, K, 5, device=dev))
+        qb = api.mx_quantize(synth.weights(N, K, 5, device=dev))
+        D = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        fn = lambda: api.mx_gemm(qa, qb, api.OUT_BF16, out=D)
+        work, unit = 2.0 * M * N * K, "TFLOP/s"
+    elif args.case == "mx_quant_row":
+        R, C = shape
+        x = synth.activations(R, C, 5, device=dev)
+        q = api.mx_quantize(x)
+        fn, work, unit = (lambda: api.mx_quantize(x, out=q)), R * C * (2 + 0.5 + 1 / 32), "GB/s"
+    elif args.case == "gemm":
         M, N, K = shape
         a_in, b_in = synth.activations(M, K, 5, device=dev), synth.weights(N, K, 5, device=dev)
         qa, _ = api.quantize(a_in, api.ROW, api.amax(a_in))
@@ -614,6 +663,7 @@ def main():
     result, tensors = run_ours(args, rank, world, device)
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, rank, world, device, tensors)
+    result["mxfp4"] = measure_mxfp4(tensors[0], tensors[1])
     del tensors
     if rank == 0 and not args.no_cpu_baseline:
         v, cores, desc, dt = oracle_sample(12.0)
