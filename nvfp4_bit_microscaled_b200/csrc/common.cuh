@@ -96,11 +96,12 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
 }
 
 // A code whose magnitude is zero is stored as +0 (0x0), never as -0 (0x8).
-// Works on eight packed nibbles at once.
+// Works on eight packed nibbles at once: adding 7 to a 3-bit magnitude sets
+// bit 3 exactly when the magnitude is non-zero, and never carries into the
+// next nibble (7 + 7 < 16), so that bit masks the sign.
 __device__ __forceinline__ uint32_t clear_negative_zero(uint32_t w) {
-  uint32_t mag = w & 0x77777777u;
-  uint32_t nz = (mag | (mag >> 1) | (mag >> 2)) & 0x11111111u;
-  return mag | (w & (nz << 3));
+  const uint32_t mag = w & 0x77777777u;
+  return mag | (w & (mag + 0x77777777u) & 0x88888888u);
 }
 
 // --------------------------------------------------------------------------

@@ -244,20 +244,26 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
 }
 
 // ---------------------------------------------------------------------------
-// 2D 16x16 (weights).  CTA tile: 64 rows (4 bands of 16, one per warp) x 512
-// columns (32 tiles, one per lane).  Pass 1 reads the tile for its maximum,
-// pass 2 re-reads it (L1-resident) and emits the codes twice: row copy
-// [N, K/2] and column copy [K, N/2] with the nibbles transposed in registers.
-// Scale words of both copies are assembled in shared memory.
+// 2D 16x16 (weights).  CTA slab: 64 rows (4 tile rows) x 128 columns (8 tile
+// columns) of W.  Warp w takes tile row w/2 and tile columns 4*(w%2) .. +3;
+// eight lanes share a tile, lane l holding columns 2*(l%8), +1 of tile l/8
+// for all 16 rows (sixteen 4-byte loads; a warp reads 128 contiguous bytes of
+// a row per load).  The tile maximum meets by shuffle; the column copy
+// [K, N/2] is stored straight from registers (16 codes = 8 bytes per column);
+// the row copy [N, K/2] gathers each row's 8 bytes per tile through a small
+// per-warp shared-memory transpose.  Row-copy scale words (4 tiles along K)
+// come from one warp; column-copy words (4 tiles along N) meet in shared
+// memory.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) quant_2d_kernel(const uint16_t* __restrict__ w, int64_t N, int64_t K,
-                                                         int64_t ld, const float* __restrict__ amax_dev,
-                                                         uint8_t* __restrict__ row_data, uint8_t* __restrict__ row_sf,
-                                                         int64_t row_sp, float* __restrict__ row_gs,
-                                                         uint8_t* __restrict__ col_data, uint8_t* __restrict__ col_sf,
-                                                         int64_t col_sp, float* __restrict__ col_gs) {
-  __shared__ uint32_t tsf[4][32];
+__global__ void __launch_bounds__(256, 4) quant_2d_kernel(const uint16_t* __restrict__ w, int64_t N, int64_t K,
+                                                           int64_t ld, const float* __restrict__ amax_dev,
+                                                           uint8_t* __restrict__ row_data, uint8_t* __restrict__ row_sf,
+                                                           int64_t row_sp, float* __restrict__ row_gs,
+                                                           uint8_t* __restrict__ col_data, uint8_t* __restrict__ col_sf,
+                                                           int64_t col_sp, float* __restrict__ col_gs) {
   __shared__ float r_tbl[kRTableSize];
+  __shared__ uint32_t tsf[4][8];
+  __shared__ __align__(16) uint8_t rowbuf[8][16][32];
   const float amax = __ldg(amax_dev);
   const float s_enc = encode_scale(amax);
   if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -266,78 +272,81 @@ __global__ void __launch_bounds__(128) quant_2d_kernel(const uint16_t* __restric
   }
   fill_r_table(r_tbl, s_enc);
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tr = warp >> 1, tq = 4 * (warp & 1), tl = lane >> 3, t8 = lane & 7;
   const int64_t TN = N >> 4, TK = K >> 4;
-  const int64_t ctas_k = (TK + 31) >> 5, ctas_n = (TN + 3) >> 2;
+  const int64_t slabs_k = (TK + 7) >> 3, slabs = ((TN + 3) >> 2) * slabs_k;
   const int64_t half_k = K >> 1, half_n = N >> 1;
+  const int64_t step = gridDim.x, step_q = step / slabs_k, step_r = step - step_q * slabs_k;
+  int64_t cn = blockIdx.x / slabs_k, ck = blockIdx.x - (blockIdx.x / slabs_k) * slabs_k;
 
-  for (int64_t ci = blockIdx.x; ci < ctas_n * ctas_k; ci += gridDim.x) {
-    const int64_t cn = ci / ctas_k, ck = ci - cn * ctas_k;
-    const int64_t bn = cn * 4 + warp, bk = ck * 32 + lane;
-    const bool ok = (bn < TN) && (bk < TK);
-    const uint16_t* tile = w + bn * 16 * ld + bk * 16;
-    uint32_t mb = 0;
-    if (ok) {
+  for (int64_t ci = blockIdx.x; ci < slabs; ci += step) {
+    const int64_t bn = cn * 4 + tr, bk = ck * 8 + tq + tl;   // this lane's tile
+    const bool row_ok = bn < TN, ok = row_ok && bk < TK;
+    const int64_t n0 = bn * 16, k0 = bk * 16 + 2 * t8;
+    uint32_t raw[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint4* src = reinterpret_cast<const uint4*>(tile + i * ld);
-        mb = max(mb, max(absmax_bits8(__ldg(src)), absmax_bits8(__ldg(src + 1))));
-      }
-    }
+    for (int i = 0; i < 16; ++i)
+      raw[i] = ok ? __ldcs(reinterpret_cast<const unsigned int*>(w + (n0 + i) * ld + k0)) : 0u;
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m2 = __vmaxu2(m2, raw[i] & 0x7FFF7FFFu);
+    uint32_t mb = max(m2 & 0xFFFFu, m2 >> 16);
+    mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 1));
+    mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 2));
+    mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 4));
     const BlockScale bs = block_scale_t(bf16_bits_to_f32(mb), s_enc, r_tbl);
-    tsf[warp][lane] = ok ? bs.sf : 0u;
-    if (ok) {
-      uint32_t colw[16][2];
+    uint32_t c0[2] = {0u, 0u}, c1[2] = {0u, 0u};
 #pragma unroll
-      for (int j = 0; j < 16; ++j) colw[j][0] = colw[j][1] = 0u;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint4* src = reinterpret_cast<const uint4*>(tile + i * ld);
-        float y[16];
-        unpack8(__ldg(src), y);
-        unpack8(__ldg(src + 1), y + 8);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) y[j] = __fmul_rn(y[j], bs.r);
-        const uint32_t w0 = pack8(y), w1 = pack8(y + 8);
-        if (row_data) *reinterpret_cast<uint2*>(row_data + (bn * 16 + i) * half_k + bk * 8) = make_uint2(w0, w1);
-        // column copy: code (i, j) becomes nibble i of column row j
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t nib = ((j < 8 ? w0 : w1) >> (4 * (j & 7))) & 0xFu;
-          colw[j][i >> 3] |= nib << (4 * (i & 7));
-        }
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t byte = f32x2_to_e2m1x2(__fmul_rn(bf16_bits_to_f32(raw[i] & 0xFFFFu), bs.r),
+                                            __fmul_rn(bf16_bits_to_f32(raw[i] >> 16), bs.r));
+      rowbuf[warp][i][tl * 8 + t8] = static_cast<uint8_t>(byte);  // negative zeros cleared per word below
+      c0[i >> 3] |= (byte & 0xFu) << (4 * (i & 7));
+      c1[i >> 3] |= (byte >> 4) << (4 * (i & 7));
+    }
+    if (ok && col_data) {
+      *reinterpret_cast<uint2*>(col_data + k0 * half_n + n0 / 2) =
+          make_uint2(clear_negative_zero(c0[0]), clear_negative_zero(c0[1]));
+      *reinterpret_cast<uint2*>(col_data + (k0 + 1) * half_n + n0 / 2) =
+          make_uint2(clear_negative_zero(c1[0]), clear_negative_zero(c1[1]));
+    }
+    const uint32_t sfv = ok ? bs.sf : 0u;
+    if (t8 == 0) tsf[tr][tq + tl] = sfv;
+    __syncwarp();
+    if (row_ok && row_data) {
+      // lane: row lane/2 of the tile row, tiles 2*(lane%2), +1 of the warp
+      const int i = lane >> 1, h = lane & 1;
+      const int64_t kt = ck * 8 + tq + 2 * h;
+      uint8_t* dst = row_data + (n0 + i) * half_k + kt * 8;
+      uint4 v = *reinterpret_cast<const uint4*>(&rowbuf[warp][i][16 * h]);
+      v = make_uint4(clear_negative_zero(v.x), clear_negative_zero(v.y), clear_negative_zero(v.z),
+                     clear_negative_zero(v.w));
+      // rows start on 8-byte boundaries (K/2 % 8 == 0), on 16-byte ones only when K/2 % 16 == 0
+      if (kt + 1 < TK && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+        *reinterpret_cast<uint4*>(dst) = v;
+      } else {
+        if (kt < TK) *reinterpret_cast<uint2*>(dst) = make_uint2(v.x, v.y);
+        if (kt + 1 < TK) *reinterpret_cast<uint2*>(dst + 8) = make_uint2(v.z, v.w);
       }
-      if (col_data) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          *reinterpret_cast<uint2*>(col_data + (bk * 16 + j) * half_n + bn * 8) = make_uint2(colw[j][0], colw[j][1]);
-      }
+    }
+    // row-copy scale word of each of the 16 rows: the warp's four tiles along K
+    uint32_t word = sfv << (8 * tl);
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 8);
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 16);
+    if (row_ok && row_sf && lane < 16 && ck * 8 + tq < TK)
+      *reinterpret_cast<uint32_t*>(row_sf + sf_offset(n0 + lane, ck * 8 + tq, row_sp)) = word;
+    __syncthreads();
+    // column-copy scale word of each of the slab's 128 columns: four tiles along N
+    if (col_sf && tid < 128 && ck * 8 + (tid >> 4) < TK) {
+      const int tc = tid >> 4;
+      const uint32_t cw = tsf[0][tc] | (tsf[1][tc] << 8) | (tsf[2][tc] << 16) | (tsf[3][tc] << 24);
+      *reinterpret_cast<uint32_t*>(col_sf + sf_offset(ck * 128 + tid, cn * 4, col_sp)) = cw;
     }
     __syncthreads();
-    // row copy scales: 64 rows x 8 words (4 tiles each)
-    if (row_sf) {
-      for (int e = threadIdx.x; e < 64 * 8; e += blockDim.x) {
-        const int band = e >> 7, i = (e >> 3) & 15, wq = e & 7;
-        const int64_t n = (cn * 4 + band) * 16 + i, kb = ck * 32 + wq * 4;
-        if (n < N && kb < TK) {
-          const uint32_t word = tsf[band][4 * wq] | (tsf[band][4 * wq + 1] << 8) | (tsf[band][4 * wq + 2] << 16) |
-                                (tsf[band][4 * wq + 3] << 24);
-          *reinterpret_cast<uint32_t*>(row_sf + sf_offset(n, kb, row_sp)) = word;
-        }
-      }
-    }
-    // column copy scales: 512 rows (k) x one word (4 bands)
-    if (col_sf) {
-      for (int e = threadIdx.x; e < 512; e += blockDim.x) {
-        const int t = e >> 4, j = e & 15;
-        const int64_t k = (ck * 32 + t) * 16 + j;
-        if (ck * 32 + t < TK) {
-          const uint32_t word = tsf[0][t] | (tsf[1][t] << 8) | (tsf[2][t] << 16) | (tsf[3][t] << 24);
-          *reinterpret_cast<uint32_t*>(col_sf + sf_offset(k, cn * 4, col_sp)) = word;
-        }
-      }
-    }
-    __syncthreads();
+    ck += step_r;
+    cn += step_q;
+    if (ck >= slabs_k) ck -= slabs_k, ++cn;
   }
 }
 
@@ -520,9 +529,9 @@ cudaError_t launch_quant_2d(const void* w, int64_t N, int64_t K, int64_t ld, con
                             void* row_data, void* row_scales, float* row_gs, void* col_data, void* col_scales,
                             float* col_gs, int num_sms, cudaStream_t s) {
   const int64_t TN = N / 16, TK = K / 16;
-  const int64_t ctas = ((TN + 3) / 4) * ((TK + 31) / 32);
-  const int grid = grid_for(ctas, 1, num_sms, 12);
-  quant_2d_kernel<<<grid, 128, 0, s>>>(static_cast<const uint16_t*>(w), N, K, ld, amax_dev,
+  const int64_t ctas = ((TN + 3) / 4) * ((TK + 7) / 8);
+  const int grid = grid_for(ctas, 1, num_sms, 16);
+  quant_2d_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(w), N, K, ld, amax_dev,
                                        static_cast<uint8_t*>(row_data), static_cast<uint8_t*>(row_scales),
                                        (TK + 3) / 4 * 4, row_gs, static_cast<uint8_t*>(col_data),
                                        static_cast<uint8_t*>(col_scales), (TN + 3) / 4 * 4, col_gs);
