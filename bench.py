@@ -332,7 +332,7 @@ def run_ours(args, rank, world, device):
         },
         "kernels": kernels,
         "roofline": {
-            "kernel": "gemm_nvf4_kernel (fprop, M=16384 N=20480 K=5120)",
+            "kernel": "gemm_fp4_pair_kernel<false> (fprop, M=16384 N=20480 K=5120)",
             "bound": "tensor",
             "achieved": round(fprop_achieved, 1),
             "peak": round(fp4_peak, 1),
