@@ -133,7 +133,9 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, nvf
  *   D[m, n] = s_gA * s_gB * sum_k dq(A[m, k]) * dq(B[n, k]),  M = A->rows,
  *   N = B->rows, K = A->cols = B->cols.
  *   D          device, [M, N] with row pitch ldd; FP32 or BF16 (out_dtype).
- * Needs K % 64 == 0, N % 16 == 0, ldd % 8 == 0, 16-byte aligned pointers.
+ * Needs K % 32 == 0 (a packed row is then a multiple of 16 bytes; a last K
+ * step of 32 is completed with zero codes and zero scales), N % 16 == 0,
+ * ldd % 8 == 0, 16-byte aligned pointers.
  */
 nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, nvfp4_out_dtype out_dtype,
                         int64_t ldd, nvfp4_stream_t stream);
@@ -154,7 +156,7 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, n
  *   round-to-nearest-even of x * 2^-s, saturating at 6.  Writes 1.0 to
  *   out->global_scale.
  * nvfp4_mx_gemm: D = sum_k dq(A[m, k]) dq(B[n, k]) on MXFP4 operands, FP32
- *   accumulation, D as in nvfp4_gemm.  Needs K % 64 == 0 and M, N multiples
+ *   accumulation, D as in nvfp4_gemm.  Needs K % 32 == 0 and M, N multiples
  *   of 256 (it runs on the CTA-pair kernel; other shapes: NVFP4_ERR_SHAPE).
  */
 size_t nvfp4_mx_scale_bytes(int64_t rows, int64_t cols);

@@ -238,6 +238,21 @@ def test_gemm_rejects_unaligned_row_stride_before_launch():
     assert (buf == 0).all()
 
 
+@pytest.mark.parametrize("M,N,K", [(256, 256, 96), (512, 256, 160), (256, 512, 288),   # CTA-pair kernel
+                                   (200, 272, 96), (130, 48, 160)])                          # single-CTA kernel
+@pytest.mark.parametrize("bf16", [False, True])
+def test_gemm_k_tail_of_32(M, N, K, bf16):
+    # K % 64 == 32: the last K=64 step is completed with zero codes (TMA fill
+    # past the row) and zero scales (scale-matrix padding)
+    xa = synth.activations(M, K, 81)
+    xb = synth.weights(N, K, 82, std=0.02)
+    qa, ca, sa, ga = _qrow(xa)
+    qb, cb, sb, gb = _qrow(xb)
+    D = api.gemm(qa, qb, api.OUT_BF16 if bf16 else api.OUT_F32)
+    D_ref, absum = O.gemm(ca, sa, ga, cb, sb, gb)
+    assert_gemm_close(D.float().cpu().numpy(), D_ref, absum, bf16=bf16, what=f"K tail {M}x{N}x{K}")
+
+
 def test_gemm_tiny_workload():
     x, w, _ = synth.workload_inputs("tiny")
     qa, ca, sa, ga = _qrow(x)

@@ -84,7 +84,7 @@ def test_argument_checks_return_before_any_launch(L):
     assert q(fake, 16, 32, 32, _lib.ROW, 0, 0, 0, fake, ctypes.byref(_t(16, 32, data=4100)), None, None) == 3
     a, b = _t(128, 256), _t(128, 256)
     assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(_t(128, 128)), fake, 0, 128, None) == 2  # K mismatch
-    assert L.nvfp4_gemm(ctypes.byref(_t(128, 96)), ctypes.byref(_t(128, 96)), fake, 0, 128, None) == 2  # K % 64
+    assert L.nvfp4_gemm(ctypes.byref(_t(128, 80)), ctypes.byref(_t(128, 80)), fake, 0, 128, None) == 2  # K % 32
     assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), fake, 7, 128, None) == 1     # bad dtype
     assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), fake + 4, 0, 128, None) == 3  # misaligned D
     assert L.nvfp4_linear_fwd(fake, fake, 100, 64, 64, fake, fake, 1 << 30, None) == 2
@@ -105,5 +105,5 @@ def test_mx_sizes_and_argument_checks(L):
     a, b = _t(256, 256), _t(256, 256)
     assert g(ctypes.byref(_t(128, 256)), ctypes.byref(b), fake, 0, 256, None) == 2   # M % 256
     assert g(ctypes.byref(a), ctypes.byref(_t(384, 256)), fake, 0, 384, None) == 2   # N % 256
-    assert g(ctypes.byref(_t(256, 96)), ctypes.byref(_t(256, 96)), fake, 0, 256, None) == 2  # K % 64
+    assert g(ctypes.byref(_t(256, 80)), ctypes.byref(_t(256, 80)), fake, 0, 256, None) == 2  # K % 32
     assert g(ctypes.byref(a), ctypes.byref(b), fake + 4, 0, 256, None) == 3        # misaligned D
