@@ -30,6 +30,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -692,6 +694,53 @@ bool make_output_map(CUtensorMap* tm, void* D, int64_t M, int64_t N, int64_t ldd
   return r == CUDA_SUCCESS;
 }
 
+// Per-device, per-kernel launch setup, done once: the dynamic shared-memory
+// opt-in (a per-device function attribute) and, for the pair kernels, how many
+// CTA pairs fit at once.  Guarded by a mutex so concurrent first calls from
+// several host threads are safe.
+struct KernelSetup {
+  bool done = false;
+  int max_pairs = 0;
+};
+
+template <class Kernel>
+cudaError_t setup_kernel(KernelSetup* cache, Kernel kern, uint32_t smem_bytes, bool cluster_pairs, int num_sms,
+                         int* max_pairs) {
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  KernelSetup& c = cache[dev];
+  if (!c.done) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes));
+    if (e != cudaSuccess) return e;
+    if (cluster_pairs) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(2 * (num_sms / 2));
+      q.blockDim = dim3(NUM_THREADS);
+      q.dynamicSmemBytes = smem_bytes;
+      cudaLaunchAttribute qa[1];
+      qa[0].id = cudaLaunchAttributeClusterDimension;
+      qa[0].val.clusterDim.x = 2;
+      qa[0].val.clusterDim.y = 1;
+      qa[0].val.clusterDim.z = 1;
+      q.attrs = qa;
+      q.numAttrs = 1;
+      int n = 0;
+      e = cudaOccupancyMaxActiveClusters(&n, kern, &q);
+      c.max_pairs = (e != cudaSuccess || n < 1) ? num_sms / 2 : n;
+      (void)cudaGetLastError();  // a failed occupancy query is not a launch error
+    }
+    c.done = true;
+  }
+  if (max_pairs) *max_pairs = c.max_pairs;
+  return cudaSuccess;
+}
+
+KernelSetup g_setup_pair_nv[64], g_setup_pair_mx[64], g_setup_single[64];
+
 }  // namespace
 
 cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a_gs, const void* b_data,
@@ -710,30 +759,11 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
   const auto* sa = static_cast<const uint8_t*>(a_scales);
   const auto* sb = static_cast<const uint8_t*>(b_scales);
   if (pair) {
-    static int max_pairs[2] = {-1, -1};
     auto kern = mx ? gemm_fp4_pair_kernel<true> : gemm_fp4_pair_kernel<false>;
-    if (max_pairs[mx ? 1 : 0] < 0) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(P_SMEM_BYTES));
-      if (e != cudaSuccess) return e;
-      cudaLaunchConfig_t q = {};
-      q.gridDim = dim3(2 * (num_sms / 2));
-      q.blockDim = dim3(NUM_THREADS);
-      q.dynamicSmemBytes = P_SMEM_BYTES;
-      cudaLaunchAttribute qa[1];
-      qa[0].id = cudaLaunchAttributeClusterDimension;
-      qa[0].val.clusterDim.x = 2;
-      qa[0].val.clusterDim.y = 1;
-      qa[0].val.clusterDim.z = 1;
-      q.attrs = qa;
-      q.numAttrs = 1;
-      int n = 0;
-      e = cudaOccupancyMaxActiveClusters(&n, kern, &q);
-      if (e != cudaSuccess || n < 1) n = num_sms / 2;
-      max_pairs[mx ? 1 : 0] = n;
-    }
+    int mp = 0;
+    cudaError_t e = setup_kernel(mx ? g_setup_pair_mx : g_setup_pair_nv, kern, P_SMEM_BYTES, true, num_sms, &mp);
+    if (e != cudaSuccess) return e;
     const int64_t tiles = (M / 256) * (N / 256);
-    const int mp = max_pairs[mx ? 1 : 0];
     const int pairs = static_cast<int>(tiles < mp ? tiles : mp);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
@@ -750,13 +780,8 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
     return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmD, sa, sb, a_gs, b_gs, static_cast<int>(M),
                               static_cast<int>(N), static_cast<int>(K), out_bf16);
   }
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(SMEM_BYTES));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = setup_kernel(g_setup_single, gemm_nvf4_kernel, SMEM_BYTES, false, num_sms, nullptr);
+  if (e != cudaSuccess) return e;
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
   gemm_nvf4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(tmA, tmB, sa, sb, a_gs, b_gs, static_cast<int>(M),
