@@ -191,3 +191,16 @@ def selftest_scale_division():
     check("nvfp4_selftest_scale_division",
           lib().nvfp4_selftest_scale_division(ctypes.byref(q), ctypes.byref(c)))
     return q.value, c.value
+
+
+# ---------------------------------------------------------------- layer precision policy
+def block_uses_bf16(block, n_blocks, first=2, last=8):
+    """Whether transformer block `block` (0-based, of n_blocks) keeps its linear
+    layers in BF16 instead of NVFP4.  "Pretraining Large Language Models with
+    NVFP4", section 2B.1: the most sensitive layers, mainly the last ones, stay
+    in high precision; the 12B run kept the first two and the last eight blocks
+    in BF16 (about 16% of the linear layers).  A host-side switch: the BF16
+    layers are the framework's own and do not go through this library."""
+    if not 0 <= block < n_blocks:
+        raise ValueError(f"block {block} outside 0..{n_blocks - 1}")
+    return block < first or block >= n_blocks - last
