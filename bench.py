@@ -479,7 +479,8 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     steps = []
-    per = max(3.0, 40.0 / max(1, args.steps + args.warmup))
+    # the whole run (warm-up and timed steps) stays near a minute whatever K and W are
+    per = max(0.2, 60.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         oracle_sample(per)
     for _ in range(args.steps):
