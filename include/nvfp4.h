@@ -156,8 +156,8 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, n
  *   round-to-nearest-even of x * 2^-s, saturating at 6.  Writes 1.0 to
  *   out->global_scale.
  * nvfp4_mx_gemm: D = sum_k dq(A[m, k]) dq(B[n, k]) on MXFP4 operands, FP32
- *   accumulation, D as in nvfp4_gemm.  Needs K % 32 == 0 and M, N multiples
- *   of 256 (it runs on the CTA-pair kernel; other shapes: NVFP4_ERR_SHAPE).
+ *   accumulation, D as in nvfp4_gemm, with the same shape rules (K % 32 == 0,
+ *   N % 16 == 0).
  */
 size_t nvfp4_mx_scale_bytes(int64_t rows, int64_t cols);
 nvfp4_status nvfp4_mx_quantize(const void* x, int64_t R, int64_t C, int64_t ld, const nvfp4_tensor* out,

@@ -147,7 +147,7 @@ nvfp4_status nvfp4_mx_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D
   if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
   const int64_t M = A->rows, N = B->rows, K = A->cols;
   if (M <= 0 || N <= 0 || K <= 0 || B->cols != K) return NVFP4_ERR_SHAPE;
-  if (K % 32 || M % 256 || N % 256 || ldd < N || M >= (1LL << 31) || N >= (1LL << 31) || K >= (1LL << 31))
+  if (K % 32 || N % 16 || ldd < N || M >= (1LL << 31) || N >= (1LL << 31) || K >= (1LL << 31))
     return NVFP4_ERR_SHAPE;
   nvfp4_status st;
   if ((st = check_tensor(A, M, K)) != NVFP4_OK || (st = check_tensor(B, N, K)) != NVFP4_OK) return st;

@@ -315,7 +315,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 }
 
 // ===========================================================================
-// CTA-pair kernel (cta_group::2) for M and N multiples of 256.
+// CTA-pair kernel (cta_group::2): every GEMM with more than 128 rows.
 //
 // A cluster of two CTAs computes a 256 x 256 tile with one pair MMA per K-step
 // (M = 256 over both CTAs' tensor memory).  Each CTA loads its own 128 rows of
@@ -401,8 +401,12 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
-  const int num_m = M / 256, num_n = N / 256;
+  // M and N need not be multiples of 256: TMA fills rows past the matrix with
+  // zeros, scale tiles past the padded scale matrix are not loaded (zeros go
+  // to tensor memory instead), and output boxes are clipped or skipped.
+  const int num_m = (M + 255) / 256, num_n = (N + 255) / 256;
   const int num_tiles = num_m * num_n;
+  const int sf_rows_a = (M + 127) / 128, sf_rows_b = (N + 127) / 128;   // 128-row scale blocks that exist
   const int katoms = (K + 63) / 64;                     // MMA steps of K = 64
   const int sf_atoms = MX ? (K + 127) / 128 : katoms;   // 128x4 scale tiles along K
   constexpr int ATOMS_PER_STAGE = MX ? KB_PER_STAGE / 2 : KB_PER_STAGE;
@@ -449,19 +453,23 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         if (!mbar_wait(&empty[stage], phase ^ 1u, kErrWaitEmpty)) { *abort_flag = 1; break; }
         const int nkb = min(KB_PER_STAGE, katoms - kt * KB_PER_STAGE);
         const uint32_t sf_bytes = static_cast<uint32_t>(MX ? (nkb + 1) / 2 : nkb) * 512u;
+        const bool a_sf = 2 * tm + static_cast<int>(rank) < sf_rows_a;
+        const bool b_sf0 = 2 * tn < sf_rows_b, b_sf1 = 2 * tn + 1 < sf_rows_b;
         if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (P_A_BYTES + P_B_BYTES));
         tma_load_2d_pair(smem + P_OFF_A + stage * P_A_BYTES, &tmA, full_l + stage * 8, kt * BK_BYTES,
                          tm * 256 + 128 * static_cast<int>(rank));
         tma_load_2d_pair(smem + P_OFF_B + stage * P_B_BYTES, &tmB, full_l + stage * 8, kt * BK_BYTES,
                          tn * 256 + 128 * static_cast<int>(rank));
-        mbar_arrive_expect_tx(&sfd_full[stage], 3 * sf_bytes);
-        bulk_load(smem + P_OFF_SFA + stage * P_SFA_BYTES,
-                  sfa + (static_cast<int64_t>(2 * tm + rank) * sf_atoms + kt * ATOMS_PER_STAGE) * 512, sf_bytes,
-                  &sfd_full[stage]);
-        for (int h = 0; h < 2; ++h)
-          bulk_load(smem + P_OFF_SFB + stage * P_SFB_BYTES + h * KB_PER_STAGE * 512,
-                    sfb + (static_cast<int64_t>(2 * tn + h) * sf_atoms + kt * ATOMS_PER_STAGE) * 512, sf_bytes,
+        mbar_arrive_expect_tx(&sfd_full[stage], (a_sf + b_sf0 + b_sf1) * sf_bytes);
+        if (a_sf)
+          bulk_load(smem + P_OFF_SFA + stage * P_SFA_BYTES,
+                    sfa + (static_cast<int64_t>(2 * tm + rank) * sf_atoms + kt * ATOMS_PER_STAGE) * 512, sf_bytes,
                     &sfd_full[stage]);
+        for (int h = 0; h < 2; ++h)
+          if (h == 0 ? b_sf0 : b_sf1)
+            bulk_load(smem + P_OFF_SFB + stage * P_SFB_BYTES + h * KB_PER_STAGE * 512,
+                      sfb + (static_cast<int64_t>(2 * tn + h) * sf_atoms + kt * ATOMS_PER_STAGE) * 512, sf_bytes,
+                      &sfd_full[stage]);
         issued[stage] = true;
         issued_parity[stage] = phase;
         if (++stage == P_STAGES) stage = 0, phase ^= 1u;
@@ -521,6 +529,12 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     int stage = 0;
     uint32_t phase = 0;
     for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
+      const int per_group = P_GROUP_M * num_n, grp = t / per_group, first_m = grp * P_GROUP_M;
+      const int gsize = min(num_m - first_m, P_GROUP_M), within = t - grp * per_group;
+      const int tm = first_m + within % gsize, tn = within / gsize;
+      // scale blocks past the padded scale matrix were not loaded: zeros instead
+      const bool a_sf = 2 * tm + static_cast<int>(rank) < sf_rows_a;
+      const bool b_sf0 = 2 * tn < sf_rows_b, b_sf1 = 2 * tn + 1 < sf_rows_b;
       bool ok = true;
       for (int kt = 0; kt < num_kt; ++kt) {
         if (!mbar_wait(&sfd_full[stage], phase, kErrWaitFull) ||
@@ -535,10 +549,12 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         uint32_t ra[16], rb[32];
 #pragma unroll
         for (int kb = 0; kb < KB_PER_STAGE; ++kb) {
-          const uint4 va = kb < natoms ? *reinterpret_cast<const uint4*>(sa + 512 * kb) : make_uint4(0, 0, 0, 0);
-          const uint4 v0 = kb < natoms ? *reinterpret_cast<const uint4*>(sb + 512 * kb) : make_uint4(0, 0, 0, 0);
-          const uint4 v1 = kb < natoms ? *reinterpret_cast<const uint4*>(sb + KB_PER_STAGE * 512 + 512 * kb)
-                                       : make_uint4(0, 0, 0, 0);
+          const uint4 va =
+              kb < natoms && a_sf ? *reinterpret_cast<const uint4*>(sa + 512 * kb) : make_uint4(0, 0, 0, 0);
+          const uint4 v0 =
+              kb < natoms && b_sf0 ? *reinterpret_cast<const uint4*>(sb + 512 * kb) : make_uint4(0, 0, 0, 0);
+          const uint4 v1 = kb < natoms && b_sf1 ? *reinterpret_cast<const uint4*>(sb + KB_PER_STAGE * 512 + 512 * kb)
+                                                : make_uint4(0, 0, 0, 0);
           ra[4 * kb + 0] = va.x; ra[4 * kb + 1] = va.y; ra[4 * kb + 2] = va.z; ra[4 * kb + 3] = va.w;
           rb[8 * kb + 0] = v0.x; rb[8 * kb + 1] = v0.y; rb[8 * kb + 2] = v0.z; rb[8 * kb + 3] = v0.w;
           rb[8 * kb + 4] = v1.x; rb[8 * kb + 5] = v1.y; rb[8 * kb + 6] = v1.z; rb[8 * kb + 7] = v1.w;
@@ -607,7 +623,7 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
+          if (lane == 0 && row0 < M && col_base + 64 * h < N) {  // boxes past the matrix: nothing to store
             tma_store_2d(&tmD, stg, col_base + 64 * h, row0);
             bulk_commit_group();
           }
@@ -632,7 +648,7 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 __fmul_rn(__uint_as_float(r[4 * j + 2]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 3]), alpha));
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
+          if (lane == 0 && row0 < M && col_base + 32 * ch < N) {
             tma_store_2d(&tmD, stg, col_base + 32 * ch, row0);
             bulk_commit_group();
           }
@@ -749,8 +765,9 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
   // The pair kernel stores through TMA: the output base must be 16-byte
   // aligned and its row stride a multiple of 16 bytes.
   const int64_t esize = out_bf16 ? 2 : 4;
-  const bool pair = (M % 256 == 0) && (N % 256 == 0) && (reinterpret_cast<uintptr_t>(D) % 16 == 0) &&
-                    ((ldd * esize) % 16 == 0);
+  // CTA pairs (256-row tiles) unless the problem has at most 128 rows, where
+  // half of every pair tile would be padding; MXFP4 always runs on them.
+  const bool pair = (mx || M > 128) && (reinterpret_cast<uintptr_t>(D) % 16 == 0) && ((ldd * esize) % 16 == 0);
   CUtensorMap tmA, tmB, tmD;
   if (!make_operand_map(&tmA, a_data, M, K, BM) || !make_operand_map(&tmB, b_data, N, K, pair ? 128 : BN))
     return cudaErrorInvalidValue;
@@ -763,7 +780,7 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
     int mp = 0;
     cudaError_t e = setup_kernel(mx ? g_setup_pair_mx : g_setup_pair_nv, kern, P_SMEM_BYTES, true, num_sms, &mp);
     if (e != cudaSuccess) return e;
-    const int64_t tiles = (M / 256) * (N / 256);
+    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const int pairs = static_cast<int>(tiles < mp ? tiles : mp);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);

@@ -72,7 +72,8 @@ def test_mx_quantize_strided_rows():
 
 
 @pytest.mark.parametrize("M,N,K", [(256, 256, 256), (512, 768, 1280), (256, 512, 64), (768, 256, 320),
-                                   (2304, 1536, 512), (256, 256, 96), (512, 256, 160)])
+                                   (2304, 1536, 512), (256, 256, 96), (512, 256, 160),
+                                   (200, 272, 320), (96, 48, 128), (1000, 528, 256)])   # M, N tails
 @pytest.mark.parametrize("bf16", [False, True])
 def test_mx_gemm_vs_oracle(M, N, K, bf16):
     xa = synth.activations(M, K, 71)

@@ -176,7 +176,7 @@ def _qrow(x, sr=False, seed=0):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 128, 256), (256, 512, 512), (200, 272, 320), (384, 256, 1024),
-                                   (130, 48, 64)])
+                                   (130, 48, 64), (1000, 1040, 320), (520, 20480 + 16, 64), (96, 400, 256)])
 @pytest.mark.parametrize("bf16", [False, True])
 def test_gemm_full_vs_oracle(M, N, K, bf16):
     xa = synth.activations(M, K, 61)
@@ -192,7 +192,7 @@ def test_gemm_full_vs_oracle(M, N, K, bf16):
                                    (2304, 1536, 512)])
 @pytest.mark.parametrize("bf16", [False, True])
 def test_gemm_cta_pair_path_vs_oracle(M, N, K, bf16):
-    # M and N multiples of 256 take the CTA-pair kernel (cta_group::2)
+    # more than 128 rows: the CTA-pair kernel (cta_group::2)
     xa = synth.activations(M, K, 63)
     xb = synth.weights(N, K, 64, std=0.02)
     qa, ca, sa, ga = _qrow(xa)
@@ -238,8 +238,9 @@ def test_gemm_rejects_unaligned_row_stride_before_launch():
     assert (buf == 0).all()
 
 
-@pytest.mark.parametrize("M,N,K", [(256, 256, 96), (512, 256, 160), (256, 512, 288),   # CTA-pair kernel
-                                   (200, 272, 96), (130, 48, 160)])                          # single-CTA kernel
+@pytest.mark.parametrize("M,N,K", [(256, 256, 96), (512, 256, 160), (256, 512, 288), (200, 272, 96),
+                                   (130, 48, 160),                                           # CTA-pair kernel
+                                   (128, 272, 96), (72, 48, 160)])                           # single-CTA kernel
 @pytest.mark.parametrize("bf16", [False, True])
 def test_gemm_k_tail_of_32(M, N, K, bf16):
     # K % 64 == 32: the last K=64 step is completed with zero codes (TMA fill

@@ -103,7 +103,7 @@ def test_mx_sizes_and_argument_checks(L):
     assert q(fake, 16, 64, 64, None, None) == 1
     g = L.nvfp4_mx_gemm
     a, b = _t(256, 256), _t(256, 256)
-    assert g(ctypes.byref(_t(128, 256)), ctypes.byref(b), fake, 0, 256, None) == 2   # M % 256
-    assert g(ctypes.byref(a), ctypes.byref(_t(384, 256)), fake, 0, 384, None) == 2   # N % 256
+    assert g(ctypes.byref(a), ctypes.byref(_t(200, 256)), fake, 0, 200, None) == 2   # N % 16
+    assert g(ctypes.byref(a), ctypes.byref(b), fake, 0, 128, None) == 2              # ldd < N
     assert g(ctypes.byref(_t(256, 80)), ctypes.byref(_t(256, 80)), fake, 0, 256, None) == 2  # K % 32
     assert g(ctypes.byref(a), ctypes.byref(b), fake + 4, 0, 256, None) == 3        # misaligned D
