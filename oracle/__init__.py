@@ -9,9 +9,11 @@ FP64 GEMM); this module only marshals numpy arrays through ctypes.  The readings
 R1..R18 (NVFP4) and R21..R24 (the MXFP4 comparison format) that fix what the
 pages leave open are listed at the top of that file.
 
-Parity unpinned: the storage layouts (R17 nibble order, R18 scale swizzle) and
-the op-order readings (R4, R6, R9, R16) have no pin in the pages; everything
-else is pinned by ``tests/test_oracle_pins.py``.
+Parity unpinned: the storage layouts (R17 nibble order, R18 scale swizzle),
+the op-order readings (R4, R6, R9, R16) and the MXFP4 scale rule and clipping
+(R23, R24: the OCP Microscaling definition the pages name but do not spell
+out) have no pin in the pages; everything else is pinned by
+``tests/test_oracle_pins.py`` and ``tests/test_oracle_mx_pins.py``.
 """
 import ctypes
 import os

@@ -53,6 +53,8 @@
  *   R24 elements: y = x * 2^-s (exact), then E2M1 round-to-nearest-even with
  *       saturation at 6 (R1, R2) -- so a block whose max is in [6*2^s, 8*2^s)
  *       clips its largest values to 6 * 2^s
+ * Parity unpinned by the pages: R23 and R24 (they name MXFP4 but do not spell
+ * out its scale rule); the tests pin them against the OCP definition only.
  * Floating point: built with -ffp-contract=off and without fast-math, so every
  * FP32 operation below is one IEEE operation in the order written.
  */
