@@ -113,17 +113,11 @@ struct u32x4 { uint32_t x, y, z, w; };
 __host__ __device__ __forceinline__ u32x4 philox4x32_10(u32x4 c, uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int round = 0; round < 10; ++round) {
-#if defined(__CUDA_ARCH__)
-    uint32_t hi0, lo0, hi1, lo1;  // one 32x32 -> 64-bit multiply each
-    asm("{\n\t.reg .b64 p;\n\tmul.wide.u32 p, %2, 0xD2511F53;\n\tmov.b64 {%1, %0}, p;\n\t}"
-        : "=r"(hi0), "=r"(lo0) : "r"(c.x));
-    asm("{\n\t.reg .b64 p;\n\tmul.wide.u32 p, %2, 0xCD9E8D57;\n\tmov.b64 {%1, %0}, p;\n\t}"
-        : "=r"(hi1), "=r"(lo1) : "r"(c.z));
-#else
-    uint64_t p0 = 0xD2511F53ull * c.x, p1 = 0xCD9E8D57ull * c.z;
-    uint32_t hi0 = static_cast<uint32_t>(p0 >> 32), lo0 = static_cast<uint32_t>(p0);
-    uint32_t hi1 = static_cast<uint32_t>(p1 >> 32), lo1 = static_cast<uint32_t>(p1);
-#endif
+    // one 32x32 -> 64-bit multiply each (a single wide multiply on the GPU);
+    // plain C so that constant counter words fold at compile time
+    const uint64_t p0 = 0xD2511F53ull * c.x, p1 = 0xCD9E8D57ull * c.z;
+    const uint32_t hi0 = static_cast<uint32_t>(p0 >> 32), lo0 = static_cast<uint32_t>(p0);
+    const uint32_t hi1 = static_cast<uint32_t>(p1 >> 32), lo1 = static_cast<uint32_t>(p1);
     c = u32x4{hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0};
     k0 += 0x9E3779B9u;
     k1 += 0xBB67AE85u;
@@ -135,8 +129,12 @@ __host__ __device__ __forceinline__ u32x4 philox4x32_10(u32x4 c, uint32_t k0, ui
 enum : uint32_t { kDomainRowSR = 0, kDomainColSR = 1, kDomainRhtSigns = 2 };
 
 // Words for the four consecutive elements 4g .. 4g+3 (row-major input index).
+// NARROW: the caller guarantees g < 2^32, so the counter's second word is a
+// compile-time 0 and, with the constant domain word, parts of the first two
+// rounds fold away (same words).
+template <bool NARROW = false>
 __device__ __forceinline__ u32x4 sr_words(uint64_t g, uint32_t domain, uint32_t k0, uint32_t k1) {
-  return philox4x32_10(u32x4{static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), domain, 0u},
+  return philox4x32_10(u32x4{static_cast<uint32_t>(g), NARROW ? 0u : static_cast<uint32_t>(g >> 32), domain, 0u},
                        k0, k1);
 }
 
@@ -153,15 +151,21 @@ __device__ __forceinline__ u32x4 sr_words(uint64_t g, uint32_t domain, uint32_t 
 // 0.5 (grid {0, 0.5}, p = 2a) the comparison (w >> 8) < a * 2^25 is done in
 // FP32 (both sides exact).  Every case is the same decision as the
 // definition above, bit for bit.
+//
+// The add-and-truncate runs on the signed bit pattern (the carry never reaches
+// the sign bit, and the mask keeps it), and without the saturation at 6: a
+// value in (6, 6.4] (the E4M3 block scale rounds to nearest, so |y| stays
+// below 6.4) comes out as 6 or 8, and the saturating E2M1 conversion turns
+// both into 6, the code the saturated value gives.
 __device__ __forceinline__ float sr_magnitude(float y, uint32_t w) {
-  const float a = fminf(fabsf(y), 6.0f);
-  const uint32_t b = __float_as_uint(a);
+  const float a = fabsf(y);
+  const uint32_t b = __float_as_uint(y);
   const bool big = a >= 1.0f;
   const uint32_t keep = big ? 0xFFC00000u : 0xFF800000u;
   const uint32_t rnd = (~w) >> (big ? 10 : 9);
   const float upper = __uint_as_float((b + rnd) & keep);
   const float lower = (__uint2float_rn(w >> 8) < __fmul_rn(a, 33554432.0f)) ? 0.5f : 0.0f;  // 2^25
-  return copysignf(a >= 0.5f ? upper : lower, y);
+  return a >= 0.5f ? upper : copysignf(lower, y);
 }
 
 // --------------------------------------------------------------------------

@@ -56,7 +56,8 @@ __device__ __forceinline__ void fwht16(float (&v)[16]) {
 // Warp item: one row segment of 32 blocks (512 elements); lane = block.
 // Scale bytes of lanes 4j..4j+3 form one 32-bit word of the 128x4 tile layout.
 // ---------------------------------------------------------------------------
-template <bool SR>
+// NARROW (SR only): every element index / 4 fits in 32 bits.
+template <bool SR, bool NARROW>
 __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
                                                           int64_t ld, const float* __restrict__ amax_dev,
                                                           uint32_t k0, uint32_t k1, uint8_t* __restrict__ data,
@@ -123,7 +124,7 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
         const uint64_t g = static_cast<uint64_t>(rr[u] * C + bb[u] * 16) >> 2;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const u32x4 w = sr_words(g + q, kDomainRowSR, k0, k1);
+          const u32x4 w = sr_words<NARROW>(g + q, kDomainRowSR, k0, k1);
           y[4 * q + 0] = sr_magnitude(y[4 * q + 0], w.x);
           y[4 * q + 1] = sr_magnitude(y[4 * q + 1], w.y);
           y[4 * q + 2] = sr_magnitude(y[4 * q + 2], w.z);
@@ -151,7 +152,7 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
 // SR word for element (t, c): Philox counter (t*C + c) >> 2, so one call
 // serves the four channels of a row.
 // ---------------------------------------------------------------------------
-template <bool RHT, bool SR>
+template <bool RHT, bool SR, bool NARROW>
 __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
                                                              int64_t ld, const float* __restrict__ amax_dev,
                                                              uint32_t sign_mask, uint32_t k0, uint32_t k1,
@@ -219,8 +220,9 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
           y1[c] = __fmul_rn(v[c][i + 1], r[c]);
         }
         if (SR) {
-          const u32x4 wa = sr_words(static_cast<uint64_t>((tbase + i) * C + c0) >> 2, kDomainColSR, k0, k1);
-          const u32x4 wb = sr_words(static_cast<uint64_t>((tbase + i + 1) * C + c0) >> 2, kDomainColSR, k0, k1);
+          const u32x4 wa = sr_words<NARROW>(static_cast<uint64_t>((tbase + i) * C + c0) >> 2, kDomainColSR, k0, k1);
+          const u32x4 wb =
+              sr_words<NARROW>(static_cast<uint64_t>((tbase + i + 1) * C + c0) >> 2, kDomainColSR, k0, k1);
           y0[0] = sr_magnitude(y0[0], wa.x); y0[1] = sr_magnitude(y0[1], wa.y);
           y0[2] = sr_magnitude(y0[2], wa.z); y0[3] = sr_magnitude(y0[3], wa.w);
           y1[0] = sr_magnitude(y1[0], wb.x); y1[1] = sr_magnitude(y1[1], wb.y);
@@ -482,9 +484,12 @@ cudaError_t launch_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, co
   auto* d = static_cast<uint8_t*>(data);
   auto* f = static_cast<uint8_t*>(scales);
   if (sr)
-    quant_row_kernel<true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+    if (R * C < (int64_t(1) << 34))  // element index / 4 fits in 32 bits
+      quant_row_kernel<true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+    else
+      quant_row_kernel<true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
   else
-    quant_row_kernel<false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+    quant_row_kernel<false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_sf_pad_zero(scales, R, S, s);
@@ -500,14 +505,19 @@ cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, co
   auto* xs = static_cast<const uint16_t*>(x);
   auto* d = static_cast<uint8_t*>(data);
   auto* f = static_cast<uint8_t*>(scales);
-  if (rht && sr)
-    quant_col_kernel<true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+  const bool narrow = R * C < (int64_t(1) << 34);  // element index / 4 fits in 32 bits
+  if (rht && sr && narrow)
+    quant_col_kernel<true, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+  else if (rht && sr)
+    quant_col_kernel<true, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
   else if (rht)
-    quant_col_kernel<true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<true, false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+  else if (sr && narrow)
+    quant_col_kernel<false, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
   else if (sr)
-    quant_col_kernel<false, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<false, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
   else
-    quant_col_kernel<false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<false, false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_sf_pad_zero(scales, C, S, s);
