@@ -95,6 +95,23 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
   return out;
 }
 
+// Eight FP32 values -> one word of eight E2M1 codes, value 2i in the low and
+// 2i+1 in the high nibble of byte i (round-to-nearest-even, saturating to 6):
+// four conversions to bytes and one vector move that assembles the word.
+__device__ __forceinline__ uint32_t f32x8_to_e2m1x8(float v0, float v1, float v2, float v3, float v4, float v5,
+                                                    float v6, float v7) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+  return out;
+}
+
 // A code whose magnitude is zero is stored as +0 (0x0), never as -0 (0x8).
 // Works on eight packed nibbles at once: adding 7 to a 3-bit magnitude sets
 // bit 3 exactly when the magnitude is non-zero, and never carries into the

@@ -23,9 +23,7 @@ namespace {
 
 // Eight scaled values -> eight nibbles, element 0 in the low nibble.
 __device__ __forceinline__ uint32_t pack8(const float* y) {
-  uint32_t w = f32x2_to_e2m1x2(y[0], y[1]) | (f32x2_to_e2m1x2(y[2], y[3]) << 8) |
-               (f32x2_to_e2m1x2(y[4], y[5]) << 16) | (f32x2_to_e2m1x2(y[6], y[7]) << 24);
-  return clear_negative_zero(w);
+  return clear_negative_zero(f32x8_to_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]));
 }
 
 __device__ __forceinline__ void unpack8(uint4 v, float* f) {
@@ -210,7 +208,6 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
         r[c] = bs.r;
         sfw[c] |= bs.sf << (8 * tb);
       }
-      uint32_t lo[4] = {0u, 0u, 0u, 0u}, hi[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int i = 0; i < 16; i += 2) {
         float y0[4], y1[4];
@@ -228,17 +225,12 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
           y1[0] = sr_magnitude(y1[0], wb.x); y1[1] = sr_magnitude(y1[1], wb.y);
           y1[2] = sr_magnitude(y1[2], wb.z); y1[3] = sr_magnitude(y1[3], wb.w);
         }
-        const int sh = 8 * ((i >> 1) & 3);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t byte = f32x2_to_e2m1x2(y0[c], y1[c]) << sh;
-          if (i < 8) lo[c] |= byte; else hi[c] |= byte;
-        }
+        for (int c = 0; c < 4; ++c) v[c][i] = y0[c], v[c][i + 1] = y1[c];  // scaled values replace the inputs
       }
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        reinterpret_cast<uint2*>(data + (c0 + c) * half_r + t0 / 2)[tb] =
-            make_uint2(clear_negative_zero(lo[c]), clear_negative_zero(hi[c]));
+        reinterpret_cast<uint2*>(data + (c0 + c) * half_r + t0 / 2)[tb] = make_uint2(pack8(v[c]), pack8(v[c] + 8));
     }
 #pragma unroll
     for (int c = 0; c < 4; ++c) *reinterpret_cast<uint32_t*>(sf + sf_offset(c0 + c, 4 * q, sp)) = sfw[c];
