@@ -178,9 +178,10 @@ __device__ __forceinline__ float sr_magnitude(float y, uint32_t w) {
   const float a = fabsf(y);
   const uint32_t b = __float_as_uint(y);
   const bool big = a >= 1.0f;
-  const uint32_t keep = big ? 0xFFC00000u : 0xFF800000u;
-  const uint32_t rnd = (~w) >> (big ? 10 : 9);
-  const float upper = __uint_as_float((b + rnd) & keep);
+  // (~w) >> sh == (2^(32-sh) - 1) - (w >> sh) == low - (w >> sh), with low
+  // the bits below the kept ones: one three-input add, no bitwise not
+  const uint32_t low = big ? 0x003FFFFFu : 0x007FFFFFu;
+  const float upper = __uint_as_float((b + low - (w >> (big ? 10 : 9))) & ~low);
   const float lower = (__uint2float_rn(w >> 8) < __fmul_rn(a, 33554432.0f)) ? 0.5f : 0.0f;  // 2^25
   return a >= 0.5f ? upper : copysignf(lower, y);
 }
