@@ -182,7 +182,8 @@ __device__ __forceinline__ float sr_magnitude(float y, uint32_t w) {
   // the bits below the kept ones: one three-input add, no bitwise not
   const uint32_t low = big ? 0x003FFFFFu : 0x007FFFFFu;
   const float upper = __uint_as_float((b + low - (w >> (big ? 10 : 9))) & ~low);
-  const float lower = (__uint2float_rn(w >> 8) < __fmul_rn(a, 33554432.0f)) ? 0.5f : 0.0f;  // 2^25
+  // below 0.5: (w >> 8) < a * 2^25 (exact) <=> (w >> 8) < ceil(a * 2^25), an integer below 2^24
+  const float lower = ((w >> 8) < __float2uint_ru(__fmul_rn(a, 33554432.0f))) ? 0.5f : 0.0f;  // 2^25
   return a >= 0.5f ? upper : copysignf(lower, y);
 }
 
