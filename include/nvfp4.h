@@ -17,7 +17,8 @@
  *    the library never allocates or frees device memory.
  *  - Work is enqueued on the caller's stream and never synchronizes the host.
  *  - Argument errors return immediately, before anything is enqueued.
- *    NVFP4_ERR_CUDA means a launch failed (cudaGetLastError is left set).
+ *    NVFP4_ERR_CUDA means a launch failed (cudaGetLastError is left set;
+ *    nvfp4_last_cuda_error() names the error).
  *  - BF16 inputs are row-major [R, C] with row pitch ld (elements), finite
  *    values only; a device pointer must be 16-byte aligned.
  *  - Per-tensor scale: amax A = max|x| (FP32), S_enc = 2688 / A to encode and
