@@ -332,7 +332,7 @@ def run_ours(args, rank, world, device):
         },
         "kernels": kernels,
         "roofline": {
-            "kernel": "gemm_fp4_pair_kernel<false> (fprop, M=16384 N=20480 K=5120)",
+            "kernel": "gemm_fp4_pair_kernel<false, false> (fprop, M=16384 N=20480 K=5120)",
             "bound": "tensor",
             "achieved": round(fprop_achieved, 1),
             "peak": round(fp4_peak, 1),
@@ -509,7 +509,7 @@ def run_reference(args, rank, world):
     }
 
 
-CASES = ("gemm", "amax", "amax_rht", "amax_both", "quant_row", "quant_row_sr", "quant_2d", "quant_col_rht",
+CASES = ("gemm", "gemm_amax", "amax", "amax_rht", "amax_both", "quant_row", "quant_row_sr", "quant_2d", "quant_col_rht",
          "quant_col_rht_sr", "mx_gemm", "mx_quant_row")
 
 
@@ -550,6 +550,39 @@ def measure_mxfp4(X, W, reps=20):
             "note": "comparison format (1x32 blocks, UE8M0 scales, no tensor scale); not part of the step"}
 
 
+def measure_epilogue_amax(X, W, rounds=4, reps=8):
+    """The fprop GEMM of the workload with the amax of Y reduced in its
+    epilogue (nvfp4_gemm_amax), against the plain GEMM followed by a separate
+    amax pass over Y: what quantizing Y for a following GEMM saves.  The three
+    are timed in turn over several rounds (medians), after the step timing."""
+    T = X.shape[0]
+    Co = W.shape[0]
+    ax, aw = api.amax(X), api.amax(W)
+    xr, _ = api.quantize(X, api.ROW, ax)
+    wr, _ = api.quantize(W, api.TWO_D, aw, col_out=False)
+    Y = torch.empty(T, Co, dtype=torch.bfloat16, device=X.device)
+    a1 = torch.empty(1, dtype=torch.float32, device=X.device)
+    a2 = torch.empty(1, dtype=torch.float32, device=X.device)
+    plain = lambda: api.gemm(xr, wr, api.OUT_BF16, out=Y)
+    fused = lambda: api.gemm_amax(xr, wr, api.OUT_BF16, out=Y, amax_out=a1)
+    sep = lambda: api.amax(Y, out=a2)
+    for _ in range(3):
+        plain(), fused(), sep()
+    torch.cuda.synchronize()
+    g, f, a = [], [], []
+    for _ in range(rounds):
+        g.append(_event_ms(plain, reps))
+        f.append(_event_ms(fused, reps))
+        a.append(_event_ms(sep, reps))
+    med = lambda v: sorted(v)[len(v) // 2]
+    g_ms, f_ms, a_ms = med(g), med(f), med(a)
+    assert float(a1.cpu()[0]) == float(a2.cpu()[0]), "epilogue amax differs from the amax pass"
+    return {"gemm_ms": round(g_ms, 4), "gemm_amax_ms": round(f_ms, 4), "amax_pass_ms": round(a_ms, 4),
+            "saved_ms": round(g_ms + a_ms - f_ms, 4),
+            "note": "fprop Y = X W^T (BF16) with max|Y| from the epilogue vs GEMM + amax pass over Y; "
+                    "not part of the step"}
+
+
 def run_case(args):
     """One kernel alone on a given shape (ncu captures, launch-shape sweeps).
     gemm: --shape M,N,K (A activations, B weights, BF16 out); the others:
@@ -572,13 +605,16 @@ def run_case(args):
         x = synth.activations(R, C, 5, device=dev)
         q = api.mx_quantize(x)
         fn, work, unit = (lambda: api.mx_quantize(x, out=q)), R * C * (2 + 0.5 + 1 / 32), "GB/s"
-    elif args.case == "gemm":
+    elif args.case in ("gemm", "gemm_amax"):
         M, N, K = shape
         a_in, b_in = synth.activations(M, K, 5, device=dev), synth.weights(N, K, 5, device=dev)
         qa, _ = api.quantize(a_in, api.ROW, api.amax(a_in))
         qb, _ = api.quantize(b_in, api.ROW, api.amax(b_in))
         D = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        fn = lambda: api.gemm(qa, qb, api.OUT_BF16, out=D)
+        if args.case == "gemm":
+            fn = lambda: api.gemm(qa, qb, api.OUT_BF16, out=D)
+        else:
+            fn = lambda: api.gemm_amax(qa, qb, api.OUT_BF16, out=D, amax_out=amax)
         work, unit = 2.0 * M * N * K, "TFLOP/s"
     else:
         R, C = shape
@@ -665,6 +701,7 @@ def main():
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, rank, world, device, tensors)
     result["mxfp4"] = measure_mxfp4(tensors[0], tensors[1])
+    result["epilogue_amax"] = measure_epilogue_amax(tensors[0], tensors[1])
     del tensors
     if rank == 0 and not args.no_cpu_baseline:
         v, cores, desc, dt = oracle_sample(12.0)

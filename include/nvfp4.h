@@ -142,6 +142,23 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, n
                         int64_t ldd, nvfp4_stream_t stream);
 
 /*
+ * nvfp4_gemm_amax -- nvfp4_gemm that also writes the per-tensor amax of its
+ * output, the first step of quantizing D for the next GEMM (section 2A of the
+ * NVFP4 page: the per-tensor scale comes from the amax of the whole tensor).
+ *   amax_dev   device, 1 float, 4-byte aligned.  Zeroed in stream order, then
+ *              set to max |D[m, n]| over the M x N outputs as stored (the
+ *              BF16 values for BF16 output), exactly: the same value
+ *              nvfp4_amax returns when run on D.  NaN outputs are not counted
+ *              (inputs are finite by contract).
+ * The epilogue reduces the maximum from the accumulator registers while it
+ * stores D, so D is not read again; pass amax_dev to nvfp4_quantize(D, ...)
+ * to skip its amax pass.  D and every shape and error rule are those of
+ * nvfp4_gemm; a null amax_dev is NVFP4_ERR_INVALID_ARG.
+ */
+nvfp4_status nvfp4_gemm_amax(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, nvfp4_out_dtype out_dtype,
+                             int64_t ldd, float* amax_dev, nvfp4_stream_t stream);
+
+/*
  * MXFP4, the format the NVFP4 page compares against ("Pretraining Large
  * Language Models with NVFP4", section 2A: blocks of 32 elements with UE8M0
  * scales instead of 16 with E4M3 scales; section 3: the 8B-model comparison).

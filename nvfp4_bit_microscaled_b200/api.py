@@ -97,6 +97,20 @@ def gemm(A, B, out_dtype=OUT_F32, out=None):
     return out
 
 
+def gemm_amax(A, B, out_dtype=OUT_BF16, out=None, amax_out=None):
+    """gemm() that also returns max|D| over the stored outputs (a 1-float
+    device tensor), reduced in the GEMM's epilogue: (D, amax)."""
+    dt = torch.float32 if out_dtype == OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty(A.rows, B.rows, dtype=dt, device=A.data.device)
+    if amax_out is None:
+        amax_out = torch.empty(1, dtype=torch.float32, device=out.device)
+    ad, bd = A.desc(), B.desc()
+    check("nvfp4_gemm_amax", lib().nvfp4_gemm_amax(ctypes.byref(ad), ctypes.byref(bd), out.data_ptr(), out_dtype,
+                                                   out.stride(0), amax_out.data_ptr(), _stream(out.device)))
+    return out, amax_out
+
+
 # ---------------------------------------------------------------- MXFP4 comparison format
 def mx_scale_bytes(rows, cols):
     return lib().nvfp4_mx_scale_bytes(rows, cols)

@@ -253,8 +253,8 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, nvf
   return NVFP4_OK;
 }
 
-nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, nvfp4_out_dtype out_dtype,
-                        int64_t ldd, nvfp4_stream_t stream) {
+static nvfp4_status gemm_checked(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, nvfp4_out_dtype out_dtype,
+                          int64_t ldd, float* amax_out, nvfp4_stream_t stream) {
   if (!A || !B || !D) return NVFP4_ERR_INVALID_ARG;
   if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
   const int64_t M = A->rows, N = B->rows, K = A->cols;
@@ -268,7 +268,19 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, n
   if ((st = device_info(&di)) != NVFP4_OK) return st;
   return cuda_status(nvfp4::launch_gemm(A->data, A->scales, A->global_scale, B->data, B->scales, B->global_scale,
                                         M, N, K, D, out_dtype == NVFP4_OUT_BF16, ldd, di.sms,
-                                        reinterpret_cast<cudaStream_t>(stream)));
+                                        reinterpret_cast<cudaStream_t>(stream), 0, amax_out));
+}
+
+nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, nvfp4_out_dtype out_dtype,
+                        int64_t ldd, nvfp4_stream_t stream) {
+  return gemm_checked(A, B, D, out_dtype, ldd, nullptr, stream);
+}
+
+nvfp4_status nvfp4_gemm_amax(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, nvfp4_out_dtype out_dtype,
+                             int64_t ldd, float* amax_dev, nvfp4_stream_t stream) {
+  if (!amax_dev) return NVFP4_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(amax_dev) % 4) return NVFP4_ERR_ALIGN;
+  return gemm_checked(A, B, D, out_dtype, ldd, amax_dev, stream);
 }
 
 size_t nvfp4_linear_workspace_bytes(int64_t T, int64_t Cin, int64_t Cout) {

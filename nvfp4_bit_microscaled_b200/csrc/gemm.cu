@@ -84,11 +84,32 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int num_m, int num_n) {
   return TileCoord{first_m + within % gsize, within / gsize};
 }
 
+// Epilogue amax.  Each thread keeps the largest |alpha * acc| of the output
+// rows it owns (rows past M are left out; columns past N hold products of
+// zero-filled B rows, so they add 0, or a NaN from padding scales, which
+// fmaxf drops).  For BF16 output the stored values are RN(v); rounding to
+// nearest is monotone and symmetric, so max |RN(v)| = RN(max |v|) and one
+// rounding of the thread's maximum gives the maximum of what it stored.
+// Non-negative floats order like their bit patterns, so a warp max on the
+// bits and one atomicMax per warp finish the reduction (the launcher zeroes
+// *amax_out first, in stream order).  The warp max names the lanes that are
+// here, so a warp whose lanes left the tile loop apart (the abort path) still
+// completes it.
+__device__ __forceinline__ void epilogue_amax_commit(float thread_max, int out_bf16, float* amax_out, int lane) {
+  if (out_bf16) thread_max = __bfloat162float(__float2bfloat16_rn(thread_max));
+  const unsigned int here = __activemask();
+  const uint32_t v = __reduce_max_sync(here, __float_as_uint(thread_max));
+  if (lane == __ffs(here) - 1 && v != 0u) atomicMax(reinterpret_cast<unsigned int*>(amax_out), v);
+}
+
+// AMAX: the epilogue also reduces max |D| over the stored outputs into
+// *amax_out (see epilogue_amax_commit).
+template <bool AMAX>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb, const float* __restrict__ gsa,
                  const float* __restrict__ gsb, int M, int N, int K, void* __restrict__ D, int out_bf16,
-                 int64_t ldd) {
+                 int64_t ldd, float* __restrict__ amax_out) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
@@ -249,12 +270,14 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const float alpha = __fmul_rn(__ldg(gsa), __ldg(gsb));
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     uint32_t acc_phase = 0;
+    float run_max = 0.0f;  // AMAX only
     for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
       const TileCoord tc = tile_coord(t, num_m, num_n);
       if (!mbar_wait(acc_full, acc_phase, kErrWaitAccFull)) { *abort_flag = 1; break; }
       tc_fence_after();
       const int row = tc.m * BM + quarter * 32 + lane;
       const int col_base = tc.n * BN + col_half * 128;
+      float tile_max = 0.0f;
       if (out_bf16) {
         // read all 128 columns (packed to BF16 pairs), release the accumulator, then store
         uint32_t packed[64];
@@ -266,8 +289,10 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
-                                                       __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
+              const float v0 = __fmul_rn(__uint_as_float(r[2 * e]), alpha);
+              const float v1 = __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha);
+              if (AMAX) tile_max = fmaxf(tile_max, fmaxf(fabsf(v0), fabsf(v1)));
+              __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
               packed[16 * ch + e] = *reinterpret_cast<uint32_t*>(&h);
             }
           }
@@ -290,6 +315,10 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           uint32_t r[32];
           tmem_ld_32x32b_x32(tmem + lane_base + ACC_COL + col_half * 128 + ch * 32, r);
           tmem_ld_wait();
+          if (AMAX) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) tile_max = fmaxf(tile_max, fabsf(__fmul_rn(__uint_as_float(r[e]), alpha)));
+          }
           if (row < M) {
             float* dst = static_cast<float*>(D) + static_cast<int64_t>(row) * ldd + col0;
 #pragma unroll
@@ -305,8 +334,10 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty);
       }
+      if (AMAX && row < M) run_max = fmaxf(run_max, tile_max);
       acc_phase ^= 1u;
     }
+    if (AMAX) epilogue_amax_commit(run_max, out_bf16, amax_out, lane);
   }
   tc_fence_before();
   __syncthreads();
@@ -379,13 +410,15 @@ __device__ __forceinline__ void pair_mma_step(uint32_t acc, uint64_t adesc, uint
 // MX selects the MXFP4 operand format: one UE8M0 scale per 32 elements, so a
 // 128x4 scale tile covers K = 128 (two MMA steps) instead of K = 64, a stage
 // carries two scale tiles per 128 rows instead of four, and each MMA step
-// names its byte pair of the scale cell (see mma_mxf4_pair).
-template <bool MX>
+// names its byte pair of the scale cell (see mma_mxf4_pair).  AMAX: the
+// epilogue also reduces max |D| into *amax_out (see epilogue_amax_commit).
+template <bool MX, bool AMAX>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmD, const uint8_t* __restrict__ sfa,
                       const uint8_t* __restrict__ sfb, const float* __restrict__ gsa,
-                      const float* __restrict__ gsb, int M, int N, int K, int out_bf16) {
+                      const float* __restrict__ gsb, int M, int N, int K, int out_bf16,
+                      float* __restrict__ amax_out) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_OFF_BAR);   // leader: A/B bytes of both CTAs
@@ -587,6 +620,7 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     uint8_t* my_row = stg + lane * 128;
     const int sw = lane & 7;
     uint32_t acc_phase = 0;
+    float run_max = 0.0f;  // AMAX only
     for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
       const int per_group = P_GROUP_M * num_n, grp = t / per_group, first_m = grp * P_GROUP_M;
       const int gsize = min(num_m - first_m, P_GROUP_M), within = t - grp * per_group;
@@ -595,6 +629,7 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       tc_fence_after();
       const int row0 = tm * 256 + 128 * static_cast<int>(rank) + quarter * 32;
       const int col_base = tn * 256 + col_half * 128;
+      float tile_max = 0.0f;
       if (out_bf16) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // two boxes of 64 columns
@@ -606,8 +641,10 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              __nv_bfloat162 v = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
-                                                       __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
+              const float v0 = __fmul_rn(__uint_as_float(r[2 * e]), alpha);
+              const float v1 = __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha);
+              if (AMAX) tile_max = fmaxf(tile_max, fmaxf(fabsf(v0), fabsf(v1)));
+              __nv_bfloat162 v = __floats2bfloat162_rn(v0, v1);
               packed[16 * ch + e] = *reinterpret_cast<uint32_t*>(&v);
             }
           }
@@ -640,6 +677,10 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty_l);
           }
+          if (AMAX) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) tile_max = fmaxf(tile_max, fabsf(__fmul_rn(__uint_as_float(r[e]), alpha)));
+          }
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
 #pragma unroll
@@ -655,8 +696,10 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
           }
         }
       }
+      if (AMAX && row0 + lane < M) run_max = fmaxf(run_max, tile_max);
       acc_phase ^= 1u;
     }
+    if (AMAX) epilogue_amax_commit(run_max, out_bf16, amax_out, lane);
     if (lane == 0) bulk_wait_all();  // stores complete before the CTA (and its shared memory) goes away
     __syncwarp();
   }
@@ -756,13 +799,14 @@ cudaError_t setup_kernel(KernelSetup* cache, Kernel kern, uint32_t smem_bytes, b
   return cudaSuccess;
 }
 
-KernelSetup g_setup_pair_nv[64], g_setup_pair_mx[64], g_setup_single[64];
+KernelSetup g_setup_pair_nv[64], g_setup_pair_mx[64], g_setup_pair_nv_amax[64], g_setup_single[64],
+    g_setup_single_amax[64];
 
 }  // namespace
 
 cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a_gs, const void* b_data,
                         const void* b_scales, const float* b_gs, int64_t M, int64_t N, int64_t K, void* D,
-                        int out_bf16, int64_t ldd, int num_sms, cudaStream_t s, int mx) {
+                        int out_bf16, int64_t ldd, int num_sms, cudaStream_t s, int mx, float* amax_out) {
   // The pair kernel stores through TMA: the output base must be 16-byte
   // aligned and its row stride a multiple of 16 bytes.
   const int64_t esize = out_bf16 ? 2 : 4;
@@ -774,12 +818,19 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
     return cudaErrorInvalidValue;
   if (pair && !make_output_map(&tmD, D, M, N, ldd, out_bf16)) return cudaErrorInvalidValue;
   if (mx && !pair) return cudaErrorInvalidValue;  // MXFP4 runs on the CTA-pair kernel only
+  if (mx && amax_out) return cudaErrorInvalidValue;  // no epilogue amax for MXFP4
   const auto* sa = static_cast<const uint8_t*>(a_scales);
   const auto* sb = static_cast<const uint8_t*>(b_scales);
+  if (amax_out) {
+    cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), s);
+    if (e != cudaSuccess) return e;
+  }
   if (pair) {
-    auto kern = mx ? gemm_fp4_pair_kernel<true> : gemm_fp4_pair_kernel<false>;
+    auto kern = mx ? gemm_fp4_pair_kernel<true, false>
+                   : (amax_out ? gemm_fp4_pair_kernel<false, true> : gemm_fp4_pair_kernel<false, false>);
+    KernelSetup* cache = mx ? g_setup_pair_mx : (amax_out ? g_setup_pair_nv_amax : g_setup_pair_nv);
     int mp = 0;
-    cudaError_t e = setup_kernel(mx ? g_setup_pair_mx : g_setup_pair_nv, kern, P_SMEM_BYTES, true, num_sms, &mp);
+    cudaError_t e = setup_kernel(cache, kern, P_SMEM_BYTES, true, num_sms, &mp);
     if (e != cudaSuccess) return e;
     const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const int pairs = static_cast<int>(tiles < mp ? tiles : mp);
@@ -796,14 +847,16 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmD, sa, sb, a_gs, b_gs, static_cast<int>(M),
-                              static_cast<int>(N), static_cast<int>(K), out_bf16);
+                              static_cast<int>(N), static_cast<int>(K), out_bf16, amax_out);
   }
-  cudaError_t e = setup_kernel(g_setup_single, gemm_nvf4_kernel, SMEM_BYTES, false, num_sms, nullptr);
+  auto kern = amax_out ? gemm_nvf4_kernel<true> : gemm_nvf4_kernel<false>;
+  cudaError_t e =
+      setup_kernel(amax_out ? g_setup_single_amax : g_setup_single, kern, SMEM_BYTES, false, num_sms, nullptr);
   if (e != cudaSuccess) return e;
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-  gemm_nvf4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(tmA, tmB, sa, sb, a_gs, b_gs, static_cast<int>(M),
-                                                         static_cast<int>(N), static_cast<int>(K), D, out_bf16, ldd);
+  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(tmA, tmB, sa, sb, a_gs, b_gs, static_cast<int>(M), static_cast<int>(N),
+                                             static_cast<int>(K), D, out_bf16, ldd, amax_out);
   return cudaGetLastError();
 }
 

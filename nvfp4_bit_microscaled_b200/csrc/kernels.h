@@ -39,10 +39,13 @@ cudaError_t launch_sf_pad_zero(void* scales, int64_t R, int64_t S, cudaStream_t 
 
 // Block-scaled FP4 GEMM: D[M,N] = sgA * sgB * sum_k A[m,k] B[n,k].  mx != 0:
 // MXFP4 operands (UE8M0 scale per 32 elements, sgA = sgB = 1 pointers still
-// read); it always runs on the CTA-pair kernel.
+// read); it always runs on the CTA-pair kernel.  amax_out (NVFP4 only): the
+// launcher zeroes *amax_out and the epilogue writes max |D| of the stored
+// values there.
 cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a_gs, const void* b_data,
                         const void* b_scales, const float* b_gs, int64_t M, int64_t N, int64_t K, void* D,
-                        int out_bf16, int64_t ldd, int num_sms, cudaStream_t s, int mx = 0);
+                        int out_bf16, int64_t ldd, int num_sms, cudaStream_t s, int mx = 0,
+                        float* amax_out = nullptr);
 
 // Bounded-wait self-test: a kernel waits on an mbarrier nobody arrives on.
 cudaError_t launch_wait_probe(uint32_t timeout_us, cudaStream_t s);

@@ -62,6 +62,10 @@ def test_fullsize_fprop_workload():
     assert_q_equal(wc, cwc, swc, aw, "W 2D col")
     Y = api.gemm(xr, wr, api.OUT_BF16)
     _check_sampled(Y, cx, sx, _gs(ax), cwr, swr, _gs(aw), True, "fprop Y", 11)
+    # the same GEMM with the amax of Y reduced in its epilogue
+    Y2, amax_y = api.gemm_amax(xr, wr, api.OUT_BF16)
+    assert torch.equal(Y2, Y)
+    assert float(amax_y.cpu()[0]) == float(Y.float().abs().max().cpu()) == float(api.amax(Y).cpu()[0])
 
 
 def test_fullsize_wgrad_workload():

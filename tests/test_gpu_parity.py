@@ -372,3 +372,54 @@ def test_wait_probe_times_out_and_reports():
     # the context is still usable afterwards
     x = synth.normal(64, 64, 1)
     assert gpu_amax(x) == O.amax(x)
+
+
+# ------------------------------------------------------------------ GEMM with epilogue amax
+@pytest.mark.parametrize("M,N,K", [(128, 128, 256), (96, 48, 128), (128, 272, 96),       # single-CTA kernel
+                                   (256, 256, 256), (200, 272, 320), (1000, 528, 256),   # CTA pairs, M/N tails
+                                   (2304, 1536, 512)])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_gemm_amax_is_max_of_stored_output(M, N, K, bf16):
+    xa = synth.activations(M, K, 91)
+    xb = synth.weights(N, K, 92, std=0.02)
+    qa, ca, sa, ga = _qrow(xa)
+    qb, cb, sb, gb = _qrow(xb)
+    out = api.OUT_BF16 if bf16 else api.OUT_F32
+    amax_buf = torch.full((1,), 1e30, dtype=torch.float32, device="cuda")   # must be overwritten
+    D, amax = api.gemm_amax(qa, qb, out, amax_out=amax_buf)
+    D_plain = api.gemm(qa, qb, out)
+    assert torch.equal(D, D_plain)                            # same outputs as nvfp4_gemm
+    got = float(amax.cpu()[0])
+    assert got == float(D.float().abs().max().cpu())          # exactly the max of what was stored
+    if bf16:
+        assert got == float(api.amax(D).cpu()[0])             # the value the amax pass would give
+    if M * N <= 1 << 20:
+        D_ref, absum = O.gemm(ca, sa, ga, cb, sb, gb)
+        assert_gemm_close(D.float().cpu().numpy(), D_ref, absum, bf16=bf16, what=f"gemm_amax {M}x{N}x{K}")
+        # and within the GEMM tolerance of the oracle's own max |D|
+        tol = 1e-4 * absum + (2.0 ** -8 * np.abs(D_ref) if bf16 else 0.0)
+        assert got <= np.max(np.abs(D_ref) + tol) and got >= np.max(np.abs(D_ref) - tol)
+
+
+def test_gemm_amax_zero_operand_and_reuse():
+    M, N, K = 256, 256, 128
+    qa, _, _, _ = _qrow(torch.zeros(M, K, dtype=torch.bfloat16))
+    qb, _, _, _ = _qrow(synth.weights(N, K, 93, std=0.02))
+    amax_buf = torch.full((1,), 5.0, dtype=torch.float32, device="cuda")
+    D, amax = api.gemm_amax(qa, qb, api.OUT_BF16, amax_out=amax_buf)
+    assert float(amax.cpu()[0]) == 0.0 and not D.any()
+    qa2, _, _, _ = _qrow(synth.activations(M, K, 94))
+    D2, amax2 = api.gemm_amax(qa2, qb, api.OUT_BF16, amax_out=amax_buf)   # same buffer, zeroed again
+    assert float(amax2.cpu()[0]) == float(D2.float().abs().max().cpu()) > 0.0
+
+
+def test_gemm_amax_feeds_the_next_quantize():
+    # the fused amax replaces the amax pass in front of quantizing D
+    M, N, K = 512, 768, 256
+    qa, _, _, _ = _qrow(synth.activations(M, K, 95))
+    qb, _, _, _ = _qrow(synth.weights(N, K, 96, std=0.02))
+    D, amax = api.gemm_amax(qa, qb, api.OUT_BF16)
+    q_fused, _ = api.quantize(D, api.ROW, amax)
+    q_pass, _ = api.quantize(D, api.ROW, api.amax(D))
+    assert torch.equal(q_fused.data, q_pass.data) and torch.equal(q_fused.scales, q_pass.scales)
+    assert torch.equal(q_fused.global_scale, q_pass.global_scale)

@@ -107,3 +107,14 @@ def test_mx_sizes_and_argument_checks(L):
     assert g(ctypes.byref(a), ctypes.byref(b), fake, 0, 128, None) == 2              # ldd < N
     assert g(ctypes.byref(_t(256, 80)), ctypes.byref(_t(256, 80)), fake, 0, 256, None) == 2  # K % 32
     assert g(ctypes.byref(a), ctypes.byref(b), fake + 4, 0, 256, None) == 3        # misaligned D
+
+
+def test_gemm_amax_argument_checks(L):
+    fake = 1 << 20
+    g = L.nvfp4_gemm_amax
+    a, b = _t(256, 256), _t(256, 256)
+    assert g(ctypes.byref(a), ctypes.byref(b), fake, 1, 256, None, None) == 1             # no amax pointer
+    assert g(ctypes.byref(a), ctypes.byref(b), fake, 1, 256, fake + 2, None) == 3         # misaligned amax
+    assert g(ctypes.byref(a), ctypes.byref(_t(200, 256)), fake, 1, 200, fake, None) == 2  # N % 16 (as nvfp4_gemm)
+    assert g(ctypes.byref(a), ctypes.byref(b), fake + 4, 1, 256, fake, None) == 3         # misaligned D
+    assert g(None, ctypes.byref(b), fake, 1, 256, fake, None) == 1
