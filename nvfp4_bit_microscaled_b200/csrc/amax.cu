@@ -68,31 +68,16 @@ __global__ void __launch_bounds__(256) amax_rows_kernel(const uint16_t* __restri
   if (lane == 0 && m) atomicMax(out, m << 16);
 }
 
-// 16-point fast Walsh-Hadamard butterflies in the fixed order h = 1, 2, 4, 8
-// (natural/Sylvester ordering: out_i = sum_j (-1)^popcount(i & j) in_j).
-__device__ __forceinline__ void fwht16(float (&v)[16]) {
-#pragma unroll
-  for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if ((j & h) == 0) {
-        float a = v[j], b = v[j + h];
-        v[j] = __fadd_rn(a, b);
-        v[j + h] = __fsub_rn(a, b);
-      }
-    }
-  }
-}
-
 // max |Q x| with Q = 1/4 * H16 * diag(s) on each aligned 16-run of rows of
 // every column (and, with BOTH, max |x| in the same pass).  Thread item: one
 // 16-row band x 4 consecutive columns: sixteen 8-byte loads, coalesced along
 // the row across the warp (256 bytes per row per warp).  The 1/4 is applied
-// after the maximum (an exact power-of-two scale commutes with max).
+// after the maximum (an exact power-of-two scale commutes with max), and the
+// transform's last butterfly stage is folded into the maximum
+// (fwht16_absmax).
 template <bool BOTH>
 __global__ void __launch_bounds__(256, 3) amax_rht_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
-                                                            int64_t ld, uint32_t sign_mask,
-                                                            unsigned int* __restrict__ out) {
+                                                            int64_t ld, unsigned int* __restrict__ out) {
   const int64_t groups = C / 4;
   const int64_t items = (R / 16) * groups;
   float m = 0.0f;
@@ -122,13 +107,10 @@ __global__ void __launch_bounds__(256, 3) amax_rht_kernel(const uint16_t* __rest
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const uint32_t word = (c < 2) ? v[i].x : v[i].y;
-        uint32_t bits = (c & 1) ? (word >> 16) : (word & 0xFFFFu);
-        bits ^= ((sign_mask >> i) & 1u) << 15;  // s_i = -1 flips the sign bit
-        f[i] = bf16_bits_to_f32(bits);
+        const float xi = __uint_as_float((c & 1) ? (word & 0xFFFF0000u) : (word << 16));
+        f[i] = rht_negates(i) ? -xi : xi;  // s_i x_i
       }
-      fwht16(f);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(f[i]));
+      m = fmaxf(m, fwht16_absmax<false>(f));
     }
   }
   m = __fmul_rn(m, 0.25f);
@@ -144,8 +126,8 @@ __global__ void __launch_bounds__(256, 3) amax_rht_kernel(const uint16_t* __rest
   }
 }
 
-cudaError_t launch_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht, uint32_t sign_mask,
-                        float* amax_dev, int num_sms, cudaStream_t s) {
+cudaError_t launch_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht, float* amax_dev, int num_sms,
+                        cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(amax_dev, 0, (rht == 2 ? 2 : 1) * sizeof(float), s);
   if (e != cudaSuccess) return e;
   if (R == 0 || C == 0) return cudaSuccess;
@@ -155,9 +137,9 @@ cudaError_t launch_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht
     const int64_t blocks = (items + 255) / 256;
     const int grid = static_cast<int>(blocks < 6LL * num_sms ? blocks : 6LL * num_sms);
     if (rht == 2)
-      amax_rht_kernel<true><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), R, C, ld, sign_mask, out);
+      amax_rht_kernel<true><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), R, C, ld, out);
     else
-      amax_rht_kernel<false><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), R, C, ld, sign_mask, out);
+      amax_rht_kernel<false><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), R, C, ld, out);
   } else if (ld == C && (R * C) % 8 == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
     const int64_t n8 = R * C / 8;
     const int64_t blocks = (n8 + 255) / 256;

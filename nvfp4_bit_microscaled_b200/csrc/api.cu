@@ -53,11 +53,6 @@ inline nvfp4_status cuda_status(cudaError_t e) {
   return NVFP4_ERR_CUDA;
 }
 
-uint32_t sign_mask() {
-  const nvfp4::u32x4 w = nvfp4::philox4x32_10(nvfp4::u32x4{0u, 0u, nvfp4::kDomainRhtSigns, 0u}, 0u, 0u);
-  return w.x & 0xFFFFu;
-}
-
 nvfp4_status check_tensor(const nvfp4_tensor* t, int64_t rows, int64_t cols) {
   if (!t || !t->data || !t->scales || !t->global_scale) return NVFP4_ERR_INVALID_ARG;
   if (t->rows != rows || t->cols != cols) return NVFP4_ERR_SHAPE;
@@ -159,7 +154,7 @@ nvfp4_status nvfp4_mx_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D
                                         reinterpret_cast<cudaStream_t>(stream), 1));
 }
 
-uint32_t nvfp4_rht_sign_mask(void) { return sign_mask(); }
+uint32_t nvfp4_rht_sign_mask(void) { return nvfp4::kRhtSignMask; }
 
 nvfp4_status nvfp4_selftest_scale_division(uint64_t* bad_quotients, uint64_t* bad_codes) {
   if (!bad_quotients || !bad_codes) return NVFP4_ERR_INVALID_ARG;
@@ -206,7 +201,7 @@ nvfp4_status nvfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht
   DeviceInfo di;
   nvfp4_status st = device_info(&di);
   if (st != NVFP4_OK) return st;
-  return cuda_status(launch_amax(x, R, C, ld, rht, sign_mask(), amax_dev, di.sms,
+  return cuda_status(launch_amax(x, R, C, ld, rht, amax_dev, di.sms,
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -246,7 +241,7 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, nvf
     if (e != cudaSuccess) return cuda_status(e);
   }
   if (want_col) {
-    e = nvfp4::launch_quant_col(x, R, C, ld, amax_dev, rht, sign_mask(), sr, seed, col_out->data,
+    e = nvfp4::launch_quant_col(x, R, C, ld, amax_dev, rht, sr, seed, col_out->data,
                                 col_out->scales, col_out->global_scale, di.sms, s);
     if (e != cudaSuccess) return cuda_status(e);
   }

@@ -127,7 +127,7 @@ __device__ __forceinline__ uint32_t clear_negative_zero(uint32_t w) {
 // --------------------------------------------------------------------------
 struct u32x4 { uint32_t x, y, z, w; };
 
-__host__ __device__ __forceinline__ u32x4 philox4x32_10(u32x4 c, uint32_t k0, uint32_t k1) {
+__host__ __device__ __forceinline__ constexpr u32x4 philox4x32_10(u32x4 c, uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int round = 0; round < 10; ++round) {
     // one 32x32 -> 64-bit multiply each (a single wide multiply on the GPU);
@@ -144,6 +144,50 @@ __host__ __device__ __forceinline__ u32x4 philox4x32_10(u32x4 c, uint32_t k0, ui
 
 // Stochastic rounding counter domains (one Philox stream per use).
 enum : uint32_t { kDomainRowSR = 0, kDomainColSR = 1, kDomainRhtSigns = 2 };
+
+// The random-sign vector s of the 16-point transform Q = 1/4 H16 diag(s),
+// fixed for the library: s_j = -1 iff bit j of word 0 of Philox(key 0,
+// counter (0, 0, kDomainRhtSigns, 0)) is set.  Evaluated at compile time, so
+// the kernels apply the signs as FP32 negations that fold into the first
+// butterfly's adds, with no per-element sign arithmetic.
+constexpr uint32_t kRhtSignMask = philox4x32_10(u32x4{0u, 0u, kDomainRhtSigns, 0u}, 0u, 0u).x & 0xFFFFu;
+__host__ __device__ __forceinline__ constexpr bool rht_negates(int j) { return ((kRhtSignMask >> j) & 1u) != 0u; }
+
+// Sylvester-order 16-point Walsh-Hadamard butterflies, stages h = 1, 2, 4, 8
+// in that order, each pair (j, j + h) with (j & h) == 0 becoming
+// (v_j + v_{j+h}, v_j - v_{j+h}) in FP32.  Returns max_j |v_j| of the result,
+// found one stage early: the last stage pairs a = v_j with b = v_{j+8}, and
+// of a + b and a - b the larger in magnitude is +-(|a| + |b|) exactly, so
+// after rounding (monotone, symmetric) max(|a + b|, |a - b|) = |a| + |b|
+// rounded: one add and one max per pair instead of two of each.  With
+// TRANSFORM = false the last stage itself is skipped (only the maximum is
+// wanted).
+template <bool TRANSFORM>
+__device__ __forceinline__ float fwht16_absmax(float (&v)[16]) {
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if ((j & h) == 0) {
+        const float a = v[j], b = v[j + h];
+        v[j] = __fadd_rn(a, b);
+        v[j + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+  float m = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) m = fmaxf(m, __fadd_rn(fabsf(v[j]), fabsf(v[j + 8])));
+  if (TRANSFORM) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float a = v[j], b = v[j + 8];
+      v[j] = __fadd_rn(a, b);
+      v[j + 8] = __fsub_rn(a, b);
+    }
+  }
+  return m;
+}
 
 // Words for the four consecutive elements 4g .. 4g+3 (row-major input index).
 // NARROW: the caller guarantees g < 2^32, so the counter's second word is a

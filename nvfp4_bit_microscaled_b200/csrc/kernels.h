@@ -5,8 +5,9 @@
 
 namespace nvfp4 {
 
-cudaError_t launch_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht, uint32_t sign_mask,
-                        float* amax_dev, int num_sms, cudaStream_t s);
+// rht: 0 max|x|, 1 max|Q x| (signs kRhtSignMask), 2 both (amax_dev[0], [1]).
+cudaError_t launch_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht, float* amax_dev, int num_sms,
+                        cudaStream_t s);
 
 // Row-wise 1x16 quantization: data [R, C/2], scales in the 128x4-tile layout
 // with sp = pad4(C/16) scale columns.
@@ -17,8 +18,8 @@ cudaError_t launch_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, co
 // Column-wise 1x16 quantization along R, optional RHT and SR; transposed
 // output data [C, R/2], scales with sp = pad4(R/16).
 cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, const float* amax_dev, int rht,
-                             uint32_t sign_mask, int sr, uint64_t seed, void* data, void* scales,
-                             float* gs_out, int num_sms, cudaStream_t s);
+                             int sr, uint64_t seed, void* data, void* scales, float* gs_out, int num_sms,
+                             cudaStream_t s);
 
 // MXFP4 row-wise 1x32 quantization: data [R, C/2], UE8M0 scales in the 128x4
 // tile layout with sp = pad4(C/32); writes 1.0 to *gs_out when given.

@@ -33,20 +33,6 @@ __device__ __forceinline__ void unpack8(uint4 v, float* f) {
   f[6] = bf16_bits_to_f32(v.w & 0xFFFFu); f[7] = bf16_bits_to_f32(v.w >> 16);
 }
 
-__device__ __forceinline__ void fwht16(float (&v)[16]) {
-#pragma unroll
-  for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if ((j & h) == 0) {
-        float a = v[j], b = v[j + h];
-        v[j] = __fadd_rn(a, b);
-        v[j + h] = __fsub_rn(a, b);
-      }
-    }
-  }
-}
-
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -153,7 +139,7 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
 template <bool RHT, bool SR, bool NARROW>
 __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
                                                              int64_t ld, const float* __restrict__ amax_dev,
-                                                             uint32_t sign_mask, uint32_t k0, uint32_t k1,
+                                                             uint32_t k0, uint32_t k1,
                                                              uint8_t* __restrict__ data, uint8_t* __restrict__ sf,
                                                              int64_t sp, float* __restrict__ gs_out) {
   __shared__ float r_tbl[kRTableSize];
@@ -186,24 +172,29 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const uint2 raw = __ldcs(reinterpret_cast<const uint2*>(x + (tbase + i) * ld + c0));
-        const uint32_t flip = RHT ? (((sign_mask >> i) & 1u) * 0x80008000u) : 0u;
-        const uint32_t a = raw.x ^ flip, b = raw.y ^ flip;
-        v[0][i] = bf16_bits_to_f32(a & 0xFFFFu);
-        v[1][i] = bf16_bits_to_f32(a >> 16);
-        v[2][i] = bf16_bits_to_f32(b & 0xFFFFu);
-        v[3][i] = bf16_bits_to_f32(b >> 16);
+        v[0][i] = __uint_as_float(raw.x << 16);
+        v[1][i] = __uint_as_float(raw.x & 0xFFFF0000u);
+        v[2][i] = __uint_as_float(raw.y << 16);
+        v[3][i] = __uint_as_float(raw.y & 0xFFFF0000u);
+        if (RHT && rht_negates(i)) {  // s_i x_i: a negation the first butterfly's adds absorb
+#pragma unroll
+          for (int c = 0; c < 4; ++c) v[c][i] = -v[c][i];
+        }
       }
       float r[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
+        float m = 0.0f;
         if (RHT) {
-          fwht16(v[c]);
+          // max |v| of the transformed run from the last butterfly's inputs;
+          // the 1/4 commutes with the maximum (exact power of two, monotone)
+          m = __fmul_rn(fwht16_absmax<true>(v[c]), 0.25f);
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[c][i] = __fmul_rn(v[c][i], 0.25f);
-        }
-        float m = 0.0f;
+        } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[c][i]));
+          for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[c][i]));
+        }
         const BlockScale bs = block_scale_t(m, s_enc, r_tbl);
         r[c] = bs.r;
         sfw[c] |= bs.sf << (8 * tb);
@@ -488,7 +479,7 @@ cudaError_t launch_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, co
 }
 
 cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, const float* amax_dev, int rht,
-                             uint32_t sign_mask, int sr, uint64_t seed, void* data, void* scales,
+                             int sr, uint64_t seed, void* data, void* scales,
                              float* gs_out, int num_sms, cudaStream_t s) {
   const int64_t S = R / 16, sp = (S + 3) / 4 * 4;
   const int64_t items = ((S + 3) / 4) * (C / 4);
@@ -499,17 +490,17 @@ cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, co
   auto* f = static_cast<uint8_t*>(scales);
   const bool narrow = R * C < (int64_t(1) << 34);  // element index / 4 fits in 32 bits
   if (rht && sr && narrow)
-    quant_col_kernel<true, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<true, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
   else if (rht && sr)
-    quant_col_kernel<true, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<true, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
   else if (rht)
-    quant_col_kernel<true, false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<true, false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
   else if (sr && narrow)
-    quant_col_kernel<false, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<false, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
   else if (sr)
-    quant_col_kernel<false, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<false, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
   else
-    quant_col_kernel<false, false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, sign_mask, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<false, false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_sf_pad_zero(scales, C, S, s);
