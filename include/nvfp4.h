@@ -129,6 +129,24 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, nvf
                             const nvfp4_tensor* col_out, nvfp4_stream_t stream);
 
 /*
+ * nvfp4_quantize_rows -- nvfp4_quantize of a block of rows of a larger tensor
+ * (one rank's token shard in data-parallel training).  x holds rows
+ * row0 .. row0 + R - 1 of a tensor with C columns; the SR word of element
+ * (r, c) of x is the one element (row0 + r, c) of the whole tensor draws,
+ * i.e. the Philox counter is ((row0 + r)*C + c) >> 2.  With the whole
+ * tensor's amax, the row copy holds the codes and scales of rows row0 .. of
+ * the whole tensor's row copy, and the column copy those of its token range
+ * row0 .. (code bytes row0/2 .., scale blocks row0/16 .. of every row), bit
+ * for bit, RN and SR alike.  row0 % 16 == 0 (a shard starts on a block
+ * boundary), 0 <= row0 < 2^40; NVFP4_2D takes row0 = 0 only
+ * (NVFP4_ERR_UNSUPPORTED otherwise).  Every other argument and error is that
+ * of nvfp4_quantize, which is this call with row0 = 0.
+ */
+nvfp4_status nvfp4_quantize_rows(const void* x, int64_t R, int64_t C, int64_t ld, nvfp4_mode mode, int rht,
+                                 int sr, uint64_t seed, int64_t row0, const float* amax_dev,
+                                 const nvfp4_tensor* row_out, const nvfp4_tensor* col_out, nvfp4_stream_t stream);
+
+/*
  * nvfp4_gemm -- block-scaled FP4 GEMM with FP32 accumulation
  * ("Como Funciona Mixed-Precision con NVFP4"; section 4 of the NVFP4 page):
  *   D[m, n] = s_gA * s_gB * sum_k dq(A[m, k]) * dq(B[n, k]),  M = A->rows,

@@ -42,6 +42,7 @@ PROTOTYPES = {
     "nvfp4_scale_bytes": (_c.c_size_t, [_i64, _i64]),
     "nvfp4_amax": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _vp]),
     "nvfp4_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _u64, _vp, _tp, _tp, _vp]),
+    "nvfp4_quantize_rows": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _u64, _i64, _vp, _tp, _tp, _vp]),
     "nvfp4_gemm": (_int, [_tp, _tp, _vp, _int, _i64, _vp]),
     "nvfp4_gemm_amax": (_int, [_tp, _tp, _vp, _int, _i64, _vp, _vp]),
     "nvfp4_linear_workspace_bytes": (_c.c_size_t, [_i64, _i64, _i64]),

@@ -64,10 +64,12 @@ def amax(x, rht=False, out=None):
     return out
 
 
-def quantize(x, mode, amax_dev, rht=False, sr=False, seed=0, row_out=None, col_out=None):
+def quantize(x, mode, amax_dev, rht=False, sr=False, seed=0, row_out=None, col_out=None, row0=0):
     """BF16 [R, C] -> (row copy, column copy); a copy the mode does not make is None.
 
     In TWO_D mode both copies are made unless row_out or col_out is False.
+    row0 != 0 (nvfp4_quantize_rows): x is rows row0 .. of a larger tensor, and
+    the SR draws are those of the whole tensor's elements.
     """
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     R, C = x.shape
@@ -79,10 +81,16 @@ def quantize(x, mode, amax_dev, rht=False, sr=False, seed=0, row_out=None, col_o
         col_out = empty_qtensor(C, R, x.device)
     rd = row_out.desc() if want_row else None
     cd = col_out.desc() if want_col else None
-    st = lib().nvfp4_quantize(x.data_ptr(), R, C, x.stride(0), mode, int(rht), int(sr), int(seed),
-                              amax_dev.data_ptr(), ctypes.byref(rd) if rd else None,
-                              ctypes.byref(cd) if cd else None, _stream(x.device))
-    check("nvfp4_quantize", st)
+    if row0:
+        st = lib().nvfp4_quantize_rows(x.data_ptr(), R, C, x.stride(0), mode, int(rht), int(sr), int(seed),
+                                       int(row0), amax_dev.data_ptr(), ctypes.byref(rd) if rd else None,
+                                       ctypes.byref(cd) if cd else None, _stream(x.device))
+        check("nvfp4_quantize_rows", st)
+    else:
+        st = lib().nvfp4_quantize(x.data_ptr(), R, C, x.stride(0), mode, int(rht), int(sr), int(seed),
+                                  amax_dev.data_ptr(), ctypes.byref(rd) if rd else None,
+                                  ctypes.byref(cd) if cd else None, _stream(x.device))
+        check("nvfp4_quantize", st)
     return (row_out if want_row else None), (col_out if want_col else None)
 
 

@@ -205,9 +205,10 @@ nvfp4_status nvfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
-nvfp4_status nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, nvfp4_mode mode, int rht, int sr,
-                            uint64_t seed, const float* amax_dev, const nvfp4_tensor* row_out,
-                            const nvfp4_tensor* col_out, nvfp4_stream_t stream) {
+static nvfp4_status quantize_checked(const void* x, int64_t R, int64_t C, int64_t ld, nvfp4_mode mode, int rht,
+                                     int sr, uint64_t seed, int64_t row0, const float* amax_dev,
+                                     const nvfp4_tensor* row_out, const nvfp4_tensor* col_out,
+                                     nvfp4_stream_t stream) {
   if (!x || !amax_dev) return NVFP4_ERR_INVALID_ARG;
   if (mode != NVFP4_ROW && mode != NVFP4_COL && mode != NVFP4_ROWCOL && mode != NVFP4_2D)
     return NVFP4_ERR_INVALID_ARG;
@@ -215,6 +216,8 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, nvf
   if (!aligned16(x) || ld % 8) return NVFP4_ERR_ALIGN;
   if (rht && mode != NVFP4_COL) return NVFP4_ERR_UNSUPPORTED;
   if (sr && mode == NVFP4_2D) return NVFP4_ERR_UNSUPPORTED;
+  if (row0 < 0 || row0 % 16 || row0 >= (int64_t(1) << 40)) return NVFP4_ERR_SHAPE;
+  if (row0 && mode == NVFP4_2D) return NVFP4_ERR_UNSUPPORTED;
   const bool want_row = mode == NVFP4_ROW || mode == NVFP4_ROWCOL || (mode == NVFP4_2D && row_out);
   const bool want_col = mode == NVFP4_COL || mode == NVFP4_ROWCOL || (mode == NVFP4_2D && col_out);
   if (mode == NVFP4_2D && !want_row && !want_col) return NVFP4_ERR_INVALID_ARG;
@@ -236,16 +239,28 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, nvf
     return cuda_status(e);
   }
   if (want_row) {
-    e = nvfp4::launch_quant_row(x, R, C, ld, amax_dev, sr, seed, row_out->data, row_out->scales,
+    e = nvfp4::launch_quant_row(x, R, C, ld, amax_dev, sr, seed, row0 * C, row_out->data, row_out->scales,
                                 row_out->global_scale, di.sms, s);
     if (e != cudaSuccess) return cuda_status(e);
   }
   if (want_col) {
-    e = nvfp4::launch_quant_col(x, R, C, ld, amax_dev, rht, sr, seed, col_out->data,
+    e = nvfp4::launch_quant_col(x, R, C, ld, amax_dev, rht, sr, seed, row0 * C, col_out->data,
                                 col_out->scales, col_out->global_scale, di.sms, s);
     if (e != cudaSuccess) return cuda_status(e);
   }
   return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, nvfp4_mode mode, int rht, int sr,
+                            uint64_t seed, const float* amax_dev, const nvfp4_tensor* row_out,
+                            const nvfp4_tensor* col_out, nvfp4_stream_t stream) {
+  return quantize_checked(x, R, C, ld, mode, rht, sr, seed, 0, amax_dev, row_out, col_out, stream);
+}
+
+nvfp4_status nvfp4_quantize_rows(const void* x, int64_t R, int64_t C, int64_t ld, nvfp4_mode mode, int rht,
+                                 int sr, uint64_t seed, int64_t row0, const float* amax_dev,
+                                 const nvfp4_tensor* row_out, const nvfp4_tensor* col_out, nvfp4_stream_t stream) {
+  return quantize_checked(x, R, C, ld, mode, rht, sr, seed, row0, amax_dev, row_out, col_out, stream);
 }
 
 static nvfp4_status gemm_checked(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D, nvfp4_out_dtype out_dtype,

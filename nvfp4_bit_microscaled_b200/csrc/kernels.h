@@ -10,16 +10,17 @@ cudaError_t launch_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht
                         cudaStream_t s);
 
 // Row-wise 1x16 quantization: data [R, C/2], scales in the 128x4-tile layout
-// with sp = pad4(C/16) scale columns.
+// with sp = pad4(C/16) scale columns.  idx0: element index of x[0][0] in the
+// tensor whose row-major index keys the SR draws (0 for a whole tensor).
 cudaError_t launch_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, const float* amax_dev, int sr,
-                             uint64_t seed, void* data, void* scales, float* gs_out, int num_sms,
+                             uint64_t seed, int64_t idx0, void* data, void* scales, float* gs_out, int num_sms,
                              cudaStream_t s);
 
 // Column-wise 1x16 quantization along R, optional RHT and SR; transposed
 // output data [C, R/2], scales with sp = pad4(R/16).
 cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, const float* amax_dev, int rht,
-                             int sr, uint64_t seed, void* data, void* scales, float* gs_out, int num_sms,
-                             cudaStream_t s);
+                             int sr, uint64_t seed, int64_t idx0, void* data, void* scales, float* gs_out,
+                             int num_sms, cudaStream_t s);
 
 // MXFP4 row-wise 1x32 quantization: data [R, C/2], UE8M0 scales in the 128x4
 // tile layout with sp = pad4(C/32); writes 1.0 to *gs_out when given.

@@ -44,9 +44,9 @@ __device__ __forceinline__ void unpack8(uint4 v, float* f) {
 template <bool SR, bool NARROW>
 __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
                                                           int64_t ld, const float* __restrict__ amax_dev,
-                                                          uint32_t k0, uint32_t k1, uint8_t* __restrict__ data,
-                                                          uint8_t* __restrict__ sf, int64_t sp,
-                                                          float* __restrict__ gs_out) {
+                                                          uint32_t k0, uint32_t k1, int64_t idx0,
+                                                          uint8_t* __restrict__ data, uint8_t* __restrict__ sf,
+                                                          int64_t sp, float* __restrict__ gs_out) {
   constexpr int U = SR ? 1 : 2;  // items in flight per warp
   __shared__ float r_tbl[kRTableSize];
   const float amax = __ldg(amax_dev);
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
 #pragma unroll
       for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(y[i], bs.r);
       if (SR) {
-        const uint64_t g = static_cast<uint64_t>(rr[u] * C + bb[u] * 16) >> 2;
+        const uint64_t g = static_cast<uint64_t>(rr[u] * C + bb[u] * 16 + idx0) >> 2;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const u32x4 w = sr_words<NARROW>(g + q, kDomainRowSR, k0, k1);
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
 template <bool RHT, bool SR, bool NARROW>
 __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
                                                              int64_t ld, const float* __restrict__ amax_dev,
-                                                             uint32_t k0, uint32_t k1,
+                                                             uint32_t k0, uint32_t k1, int64_t idx0,
                                                              uint8_t* __restrict__ data, uint8_t* __restrict__ sf,
                                                              int64_t sp, float* __restrict__ gs_out) {
   __shared__ float r_tbl[kRTableSize];
@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
   const int64_t ng = C >> 2;
   const int64_t items = nq * ng;
   const int64_t half_r = R >> 1;
+  const uint64_t cq = static_cast<uint64_t>(C) >> 2;
   // item it = (token quad it / ng, channel group it % ng), kept incrementally
   const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x, step_q = step / ng, step_r = step - step_q * ng;
@@ -168,6 +169,9 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
     uint32_t sfw[4] = {0u, 0u, 0u, 0u};
     for (int tb = 0; tb < nb; ++tb) {
       const int64_t tbase = t0 + 16 * tb;
+      // SR counter of (tbase, c0): its element index in the whole tensor / 4
+      // (C, c0 and idx0 are multiples of 4, so row i adds i * C/4 exactly)
+      const uint64_t gq = static_cast<uint64_t>(tbase * C + c0 + idx0) >> 2;
       float v[4][16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -208,9 +212,8 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
           y1[c] = __fmul_rn(v[c][i + 1], r[c]);
         }
         if (SR) {
-          const u32x4 wa = sr_words<NARROW>(static_cast<uint64_t>((tbase + i) * C + c0) >> 2, kDomainColSR, k0, k1);
-          const u32x4 wb =
-              sr_words<NARROW>(static_cast<uint64_t>((tbase + i + 1) * C + c0) >> 2, kDomainColSR, k0, k1);
+          const u32x4 wa = sr_words<NARROW>(gq + i * cq, kDomainColSR, k0, k1);
+          const u32x4 wb = sr_words<NARROW>(gq + (i + 1) * cq, kDomainColSR, k0, k1);
           y0[0] = sr_magnitude(y0[0], wa.x); y0[1] = sr_magnitude(y0[1], wa.y);
           y0[2] = sr_magnitude(y0[2], wa.z); y0[3] = sr_magnitude(y0[3], wa.w);
           y1[0] = sr_magnitude(y1[0], wb.x); y1[1] = sr_magnitude(y1[1], wb.y);
@@ -457,7 +460,7 @@ static inline int grid_for(int64_t work_units, int per_block, int num_sms, int w
 }
 
 cudaError_t launch_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, const float* amax_dev, int sr,
-                             uint64_t seed, void* data, void* scales, float* gs_out, int num_sms,
+                             uint64_t seed, int64_t idx0, void* data, void* scales, float* gs_out, int num_sms,
                              cudaStream_t s) {
   const int64_t S = C / 16, sp = (S + 3) / 4 * 4;
   const int64_t warp_items = R * ((S + 31) / 32);
@@ -467,20 +470,20 @@ cudaError_t launch_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, co
   auto* d = static_cast<uint8_t*>(data);
   auto* f = static_cast<uint8_t*>(scales);
   if (sr)
-    if (R * C < (int64_t(1) << 34))  // element index / 4 fits in 32 bits
-      quant_row_kernel<true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+    if (idx0 + R * C < (int64_t(1) << 34))  // element index / 4 fits in 32 bits
+      quant_row_kernel<true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
     else
-      quant_row_kernel<true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+      quant_row_kernel<true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else
-    quant_row_kernel<false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+    quant_row_kernel<false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_sf_pad_zero(scales, R, S, s);
 }
 
 cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, const float* amax_dev, int rht,
-                             int sr, uint64_t seed, void* data, void* scales,
-                             float* gs_out, int num_sms, cudaStream_t s) {
+                             int sr, uint64_t seed, int64_t idx0, void* data, void* scales, float* gs_out,
+                             int num_sms, cudaStream_t s) {
   const int64_t S = R / 16, sp = (S + 3) / 4 * 4;
   const int64_t items = ((S + 3) / 4) * (C / 4);
   const int grid = grid_for(items, 256, num_sms, 8);
@@ -488,19 +491,19 @@ cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, co
   auto* xs = static_cast<const uint16_t*>(x);
   auto* d = static_cast<uint8_t*>(data);
   auto* f = static_cast<uint8_t*>(scales);
-  const bool narrow = R * C < (int64_t(1) << 34);  // element index / 4 fits in 32 bits
+  const bool narrow = idx0 + R * C < (int64_t(1) << 34);  // element index / 4 fits in 32 bits
   if (rht && sr && narrow)
-    quant_col_kernel<true, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<true, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else if (rht && sr)
-    quant_col_kernel<true, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<true, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else if (rht)
-    quant_col_kernel<true, false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<true, false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else if (sr && narrow)
-    quant_col_kernel<false, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<false, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else if (sr)
-    quant_col_kernel<false, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<false, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else
-    quant_col_kernel<false, false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, d, f, sp, gs_out);
+    quant_col_kernel<false, false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_sf_pad_zero(scales, C, S, s);

@@ -1,0 +1,86 @@
+"""Data-parallel NVFP4 linear layer: tokens sharded over the ranks of a
+torch.distributed process group (NCCL on GPUs), the weight replicated.
+
+A DP training step of Y = X W^T needs two exchanges beyond the single-GPU
+path ("Pretraining Large Language Models with NVFP4", sections 2A and 2B):
+
+- the per-tensor scale of X, Q.X, dY and Q.dY comes from the amax of the
+  whole batch (two-level scaling), so each pass all-reduces (MAX) its local
+  amaxes, two floats in one collective, before any quantize kernel runs;
+- the partial FP32 weight gradients of the ranks are summed (all-reduce SUM).
+
+Stochastic rounding draws are keyed by the element's index in the whole
+batch (nvfp4_quantize_rows with row0 = rank * T_local), so every rank's
+quantized copies are the matching slices of a one-GPU quantization of the
+whole batch, bit for bit, and Y and dX are the matching rows of the one-GPU
+outputs.  Only dW differs from the one-GPU result, by the order of the final
+FP32 sum.  W is replicated, so its amax needs no exchange.
+
+Every computation runs in libnvfp4.so; this module only sequences the calls
+and the collectives.
+"""
+import torch
+import torch.distributed as dist
+
+from . import api
+
+
+class DataParallelLinear:
+    """One linear layer's forward and backward on this rank's T_local tokens.
+
+    The quantized operands live in buffers owned by the object (the same
+    operands nvfp4_linear_fwd keeps in its workspace); forward() must run
+    before backward() for the same batch.
+    """
+
+    def __init__(self, T_local, Cin, Cout, device, group=None):
+        if T_local % 16 or Cin % 16 or Cout % 16:
+            raise ValueError("T_local, Cin and Cout must be multiples of 16")
+        self.group = group
+        self.rank = dist.get_rank(group) if dist.is_initialized() else 0
+        self.world = dist.get_world_size(group) if dist.is_initialized() else 1
+        self.T, self.Cin, self.Cout = T_local, Cin, Cout
+        self.row0 = self.rank * T_local
+        dev = torch.device(device)
+        q = api.empty_qtensor
+        self.x_row, self.x_col = q(T_local, Cin, dev), q(Cin, T_local, dev)
+        self.w_row, self.w_col = q(Cout, Cin, dev), q(Cin, Cout, dev)
+        self.dy_row, self.dy_col = q(T_local, Cout, dev), q(Cout, T_local, dev)
+        self.amax_x = torch.zeros(2, dtype=torch.float32, device=dev)   # [max|X|, max|Q X|]
+        self.amax_w = torch.zeros(1, dtype=torch.float32, device=dev)
+        self.amax_dy = torch.zeros(2, dtype=torch.float32, device=dev)  # [max|dY|, max|Q dY|]
+
+    def _all_reduce(self, t, op):
+        if self.world == 1:
+            return
+        if t.is_cuda and dist.get_backend(self.group) == "gloo":
+            # gloo reduces host memory: stage through it (NCCL reduces in place on the device)
+            h = t.cpu()
+            dist.all_reduce(h, op=op, group=self.group)
+            t.copy_(h)
+        else:
+            dist.all_reduce(t, op=op, group=self.group)
+
+    def forward(self, X, W, Y=None):
+        """Y[T_local, Cout] = X W^T (BF16) for this rank's tokens."""
+        assert X.shape == (self.T, self.Cin) and W.shape == (self.Cout, self.Cin)
+        api.amax(X, rht=2, out=self.amax_x)
+        self._all_reduce(self.amax_x, dist.ReduceOp.MAX)
+        api.amax(W, out=self.amax_w)
+        api.quantize(X, api.ROW, self.amax_x[0:1], row_out=self.x_row, row0=self.row0)
+        api.quantize(W, api.TWO_D, self.amax_w, row_out=self.w_row, col_out=self.w_col)
+        api.quantize(X, api.COL, self.amax_x[1:2], rht=True, col_out=self.x_col, row0=self.row0)
+        return api.gemm(self.x_row, self.w_row, api.OUT_BF16, out=Y)
+
+    def backward(self, dY, seed, dX=None, dW=None):
+        """(dX[T_local, Cin] BF16, dW[Cout, Cin] FP32 summed over the ranks)."""
+        assert dY.shape == (self.T, self.Cout)
+        api.amax(dY, rht=2, out=self.amax_dy)
+        self._all_reduce(self.amax_dy, dist.ReduceOp.MAX)
+        api.quantize(dY, api.ROW, self.amax_dy[0:1], sr=True, seed=seed, row_out=self.dy_row, row0=self.row0)
+        api.quantize(dY, api.COL, self.amax_dy[1:2], rht=True, sr=True, seed=seed, col_out=self.dy_col,
+                     row0=self.row0)
+        dX = api.gemm(self.dy_row, self.w_col, api.OUT_BF16, out=dX)
+        dW = api.gemm(self.dy_col, self.x_col, api.OUT_F32, out=dW)
+        self._all_reduce(dW, dist.ReduceOp.SUM)
+        return dX, dW

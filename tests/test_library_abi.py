@@ -118,3 +118,15 @@ def test_gemm_amax_argument_checks(L):
     assert g(ctypes.byref(a), ctypes.byref(_t(200, 256)), fake, 1, 200, fake, None) == 2  # N % 16 (as nvfp4_gemm)
     assert g(ctypes.byref(a), ctypes.byref(b), fake + 4, 1, 256, fake, None) == 3         # misaligned D
     assert g(None, ctypes.byref(b), fake, 1, 256, fake, None) == 1
+
+
+def test_quantize_rows_argument_checks(L):
+    fake = 1 << 20
+    q = L.nvfp4_quantize_rows
+    row, col = _t(32, 64), _t(64, 32)
+    assert q(fake, 32, 64, 64, _lib.ROW, 0, 1, 0, 8, fake, ctypes.byref(row), None, None) == 2     # row0 % 16
+    assert q(fake, 32, 64, 64, _lib.ROW, 0, 1, 0, -16, fake, ctypes.byref(row), None, None) == 2   # row0 < 0
+    assert q(fake, 32, 64, 64, _lib.COL, 1, 1, 0, 1 << 40, fake, None, ctypes.byref(col), None) == 2  # too far
+    assert q(fake, 32, 64, 64, _lib.TWO_D, 0, 0, 0, 16, fake, ctypes.byref(row), ctypes.byref(col), None) == 4
+    assert q(fake, 32, 64, 64, _lib.ROW, 1, 1, 0, 16, fake, ctypes.byref(row), None, None) == 4    # RHT on rows
+    assert q(None, 32, 64, 64, _lib.ROW, 0, 1, 0, 16, fake, ctypes.byref(row), None, None) == 1
