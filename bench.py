@@ -610,11 +610,13 @@ def run_case(args):
         a_in, b_in = synth.activations(M, K, 5, device=dev), synth.weights(N, K, 5, device=dev)
         qa, _ = api.quantize(a_in, api.ROW, api.amax(a_in))
         qb, _ = api.quantize(b_in, api.ROW, api.amax(b_in))
-        D = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        f32 = args.out == "f32"
+        D = torch.empty(M, N, dtype=torch.float32 if f32 else torch.bfloat16, device=dev)
+        od = api.OUT_F32 if f32 else api.OUT_BF16
         if args.case == "gemm":
-            fn = lambda: api.gemm(qa, qb, api.OUT_BF16, out=D)
+            fn = lambda: api.gemm(qa, qb, od, out=D)
         else:
-            fn = lambda: api.gemm_amax(qa, qb, api.OUT_BF16, out=D, amax_out=amax)
+            fn = lambda: api.gemm_amax(qa, qb, od, out=D, amax_out=amax)
         work, unit = 2.0 * M * N * K, "TFLOP/s"
     else:
         R, C = shape
@@ -644,22 +646,39 @@ def run_case(args):
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(args.steps):
-        fn()
-    e.record()
-    torch.cuda.synchronize()
-    ms = s.elapsed_time(e) / args.steps
+    if args.flush:
+        # inputs that fit in L2 would be re-read from it: evict between launches, time each launch alone
+        scratch = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for s, e in evs:
+            scratch.fill_(1)
+            s.record()
+            fn()
+            e.record()
+        torch.cuda.synchronize()
+        ms = sum(s.elapsed_time(e) for s, e in evs) / args.steps
+    else:
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(args.steps):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        ms = s.elapsed_time(e) / args.steps
     rate = work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
-    print(json.dumps({"case": args.case, "shape": shape, "ms_per_launch": round(ms, 4),
-                      "rate": round(rate, 1), "unit": unit}), flush=True)
+    print(json.dumps({"case": args.case, "shape": shape, "out": args.out if "gemm" in args.case else None,
+                      "flush": bool(args.flush), "ms_per_launch": round(ms, 4), "rate": round(rate, 1),
+                      "unit": unit}), flush=True)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--case", choices=CASES, help="time one kernel alone on --shape")
     ap.add_argument("--shape", default="")
+    ap.add_argument("--out", choices=["bf16", "f32"], default="bf16", help="--case gemm: output type")
+    ap.add_argument("--flush", action="store_true",
+                    help="--case: write a 256 MiB buffer (twice L2) before each launch and time launches one by one")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
