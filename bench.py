@@ -310,13 +310,7 @@ def run_ours(args, rank, world, device):
         "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, fp32 accumulate)",
         "data": "synthetic (seeded; X ~ N(0,1) with 0.1% outlier channels x100, W ~ N(0,0.02), "
                 "dY ~ N(0,1e-3) x per-row lognormal)",
-        "config": {
-            "workload": f"full linear fwd+bwd: T={T}, Cin={Ci}, Cout={Co} (FFN up-projection of a 12B hybrid "
-                        f"Mamba-Transformer); 3 GEMMs, 3 amax, 5 quantize kernels per step",
-            "T": T, "Cin": Ci, "Cout": Co,
-            "parallelism": f"independent batch per GPU x{world}",
-            "l2": "inputs larger than L2 (X 168 MB, W 210 MB, dY 671 MB; L2 126 MB): no flush needed",
-        },
+        "config": workload_config(world),
         "gemm": {
             "tflops_gemm_only": round(sum(gf.values()) / (g_ms * 1e-3) / 1e12, 1),
             "frac_fp4_peak": round(sum(gf.values()) / (g_ms * 1e-3) / 1e12 / fp4_peak, 4),
@@ -475,6 +469,18 @@ def oracle_sample(seconds_target=15.0):
     return flops / dt / 1e12, O.num_threads(), desc, dt
 
 
+def workload_config(world):
+    """The config object both arms print: the full linear layer's workload."""
+    T, Ci, Co = WORKLOAD["T"], WORKLOAD["Cin"], WORKLOAD["Cout"]
+    return {
+        "workload": f"full linear fwd+bwd: T={T}, Cin={Ci}, Cout={Co} (FFN up-projection of a 12B hybrid "
+                    f"Mamba-Transformer); 3 GEMMs, 3 amax, 5 quantize kernels per step",
+        "T": T, "Cin": Ci, "Cout": Co,
+        "parallelism": f"independent batch per GPU x{world}",
+        "l2": "inputs larger than L2 (X 168 MB, W 210 MB, dY 671 MB; L2 126 MB): no flush needed",
+    }
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -502,8 +508,7 @@ def run_reference(args, rank, world):
         "vs_baseline": None,
         "dtype": "f64 GEMM on fp32-quantized operands",
         "data": "synthetic (seeded)",
-        "config": {"workload": f"full linear fwd+bwd: T={WORKLOAD['T']}, Cin={WORKLOAD['Cin']}, "
-                               f"Cout={WORKLOAD['Cout']} (bounded sample, see cpu_baseline)"},
+        "config": workload_config(world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
