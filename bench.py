@@ -22,6 +22,7 @@ import re
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import torch
@@ -74,7 +75,7 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu_index = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"nvfp4_bench_clocks_{os.getpid()}_{gpu_index}.csv")
         self.t0 = self.t1 = None
 
     def mark_start(self):
