@@ -138,7 +138,8 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, nvf
  * the whole tensor's row copy, and the column copy those of its token range
  * row0 .. (code bytes row0/2 .., scale blocks row0/16 .. of every row), bit
  * for bit, RN and SR alike.  row0 % 16 == 0 (a shard starts on a block
- * boundary), 0 <= row0 < 2^40; NVFP4_2D takes row0 = 0 only
+ * boundary), 0 <= row0 < 2^40 and (row0 + R) * C < 2^62 (NVFP4_ERR_SHAPE
+ * otherwise); NVFP4_2D takes row0 = 0 only
  * (NVFP4_ERR_UNSUPPORTED otherwise).  Every other argument and error is that
  * of nvfp4_quantize, which is this call with row0 = 0.
  */

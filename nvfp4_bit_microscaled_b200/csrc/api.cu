@@ -217,6 +217,7 @@ static nvfp4_status quantize_checked(const void* x, int64_t R, int64_t C, int64_
   if (rht && mode != NVFP4_COL) return NVFP4_ERR_UNSUPPORTED;
   if (sr && mode == NVFP4_2D) return NVFP4_ERR_UNSUPPORTED;
   if (row0 < 0 || row0 % 16 || row0 >= (int64_t(1) << 40)) return NVFP4_ERR_SHAPE;
+  if (row0 && row0 + R > (int64_t(1) << 62) / C) return NVFP4_ERR_SHAPE;  // (row0 + R) * C stays in int64
   if (row0 && mode == NVFP4_2D) return NVFP4_ERR_UNSUPPORTED;
   const bool want_row = mode == NVFP4_ROW || mode == NVFP4_ROWCOL || (mode == NVFP4_2D && row_out);
   const bool want_col = mode == NVFP4_COL || mode == NVFP4_ROWCOL || (mode == NVFP4_2D && col_out);

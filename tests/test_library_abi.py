@@ -130,3 +130,5 @@ def test_quantize_rows_argument_checks(L):
     assert q(fake, 32, 64, 64, _lib.TWO_D, 0, 0, 0, 16, fake, ctypes.byref(row), ctypes.byref(col), None) == 4
     assert q(fake, 32, 64, 64, _lib.ROW, 1, 1, 0, 16, fake, ctypes.byref(row), None, None) == 4    # RHT on rows
     assert q(None, 32, 64, 64, _lib.ROW, 0, 1, 0, 16, fake, ctypes.byref(row), None, None) == 1
+    wide = _t(32, 1 << 24)
+    assert q(fake, 32, 1 << 24, 1 << 24, _lib.ROW, 0, 1, 0, 1 << 39, fake, ctypes.byref(wide), None, None) == 2  # index overflow
