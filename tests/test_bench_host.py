@@ -1,0 +1,83 @@
+"""Host-side logic of bench.py, CPU only: the clock record that decides whether
+a run is kept (samples outside the timed region ignored, throttle reasons
+collected, median clock), the GEMM traffic figure that is reported only while
+the kernel source still matches the ncu capture, and the config object both
+arms print."""
+import datetime
+import hashlib
+import os
+import re
+
+import bench
+
+
+def _line(ts, sm, reasons=("Not Active",) * 4):
+    stamp = datetime.datetime.fromtimestamp(ts).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+    return ", ".join([stamp, "0", str(sm), "1965", "990.0", "0x0000000000000004", *reasons]) + "\n"
+
+
+def test_clock_summary_keeps_timed_samples_and_reasons(tmp_path):
+    c = bench.ClockSampler(0)
+    c.path = str(tmp_path / "clocks.csv")
+    c.proc = object()                          # as if nvidia-smi had been started
+    t0 = 1_800_000_000.0
+    c.t0, c.t1 = t0, t0 + 10.0
+    with open(c.path, "w") as f:
+        f.write(_line(t0 - 5.0, 600, ("Active",) * 4))                 # before the timed region
+        f.write(_line(t0 + 1.0, 1700))
+        f.write(_line(t0 + 2.0, 1650, ("Not Active", "Not Active", "Not Active", "Active")))
+        f.write(_line(t0 + 3.0, 1750))
+        f.write("garbage line\n")
+        f.write(_line(t0 + 20.0, 300, ("Active",) * 4))                # after it
+    s = c.summary()
+    assert s["samples"] == 3 and s["sm_mhz"] == 1700 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"]
+    assert not os.path.exists(c.path)
+
+
+def test_clock_summary_flags_hardware_slowdown(tmp_path):
+    c = bench.ClockSampler(0)
+    c.path = str(tmp_path / "clocks.csv")
+    c.proc = object()
+    t0 = 1_800_000_000.0
+    c.t0, c.t1 = t0, t0 + 10.0
+    with open(c.path, "w") as f:
+        f.write(_line(t0 + 1.0, 1200, ("Active", "Not Active", "Active", "Not Active")))
+    s = c.summary()
+    assert s["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+
+
+def test_clock_summary_without_samples(tmp_path):
+    c = bench.ClockSampler(0)
+    assert c.summary()["reasons"] == ["nvidia-smi unavailable"]
+    c.path = str(tmp_path / "empty.csv")
+    c.proc = object()
+    open(c.path, "w").close()
+    assert c.summary()["reasons"] == ["no samples"]
+
+
+def test_gemm_traffic_is_reported_only_for_the_profiled_source(tmp_path, monkeypatch):
+    root = tmp_path
+    (root / "profiles").mkdir()
+    (root / "nvfp4_bit_microscaled_b200" / "csrc").mkdir(parents=True)
+    src = b"// kernel source\n"
+    (root / "nvfp4_bit_microscaled_b200" / "csrc" / "gemm.cu").write_bytes(src)
+    prof = root / "profiles" / "gemm_nvf4_full.md"
+    prof.write_text(f"traffic_bytes_per_launch: 1234567\ngemm_source_sha256: {hashlib.sha256(src).hexdigest()}\n")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.gemm_traffic_from_profile() == 1234567.0
+    (root / "nvfp4_bit_microscaled_b200" / "csrc" / "gemm.cu").write_bytes(src + b"// changed\n")
+    assert bench.gemm_traffic_from_profile() is None
+
+
+def test_committed_gemm_profile_parses():
+    text = open(os.path.join(bench.ROOT, "profiles", "gemm_nvf4_full.md")).read()
+    assert re.search(r"traffic_bytes_per_launch:\s*[0-9]+", text)
+    assert re.search(r"gemm_source_sha256:\s*[0-9a-f]{64}", text)
+
+
+def test_both_arms_print_the_same_config():
+    c1, c8 = bench.workload_config(1), bench.workload_config(8)
+    assert c1["T"] == bench.WORKLOAD["T"] and c1["Cin"] == bench.WORKLOAD["Cin"]
+    assert c1["Cout"] == bench.WORKLOAD["Cout"]
+    assert c8["parallelism"].endswith("x8") and c1["workload"] == c8["workload"]
