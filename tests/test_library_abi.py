@@ -132,3 +132,23 @@ def test_quantize_rows_argument_checks(L):
     assert q(None, 32, 64, 64, _lib.ROW, 0, 1, 0, 16, fake, ctypes.byref(row), None, None) == 1
     wide = _t(32, 1 << 24)
     assert q(fake, 32, 1 << 24, 1 << 24, _lib.ROW, 0, 1, 0, 1 << 39, fake, ctypes.byref(wide), None, None) == 2  # index overflow
+
+
+def test_valid_calls_without_a_gpu_fail_loudly(L):
+    # every argument is valid, so the call gets as far as asking CUDA for the
+    # device: on a machine without one it must return an error, never compute
+    # on the host (there is no fallback path)
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present: this checks the no-GPU behaviour")
+    buf = ctypes.create_string_buffer((1 << 17) + 16)  # room for every operand below, D included
+    base = (ctypes.addressof(buf) + 15) // 16 * 16
+    st = L.nvfp4_amax(base, 16, 32, 32, 0, base + 4096, None)
+    assert st in (5, 6)                                    # NVFP4_ERR_DEVICE / NVFP4_ERR_CUDA
+    q = L.nvfp4_quantize
+    row = _lib.Nvfp4Tensor(base + 8192, base + 16384, base + 32768, 16, 32)
+    assert q(base, 16, 32, 32, _lib.ROW, 0, 0, 0, base + 4096, ctypes.byref(row), None, None) in (5, 6)
+    a = _lib.Nvfp4Tensor(base + 8192, base + 16384, base + 32768, 128, 64)
+    assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(a), base + 65536, 0, 128, None) in (5, 6)
+    with pytest.raises(_lib.Nvfp4Error):
+        _lib.check("nvfp4_amax", L.nvfp4_amax(base, 16, 32, 32, 0, base + 4096, None))
