@@ -232,13 +232,18 @@ nvfp4_status nvfp4_linear_bwd(const void* dY, int64_t T, int64_t Cin, int64_t Co
  * every device allocation.  Instead of a caller workspace it uses one scratch
  * area of NVFP4_NOALLOC_SCRATCH_BYTES inside the library image (a __device__
  * array that every GPU which loads the library holds until process exit).
- *   - Computes exactly what nvfp4_linear_fwd computes (same kernels, same
- *     order); Y is written as there.  X, W, Y as in nvfp4_linear_fwd.
- *   - Returns NVFP4_ERR_WORKSPACE, before enqueuing anything, when
- *     nvfp4_linear_workspace_bytes(T, Cin, Cout) exceeds the scratch size.
+ *   - Computes Y exactly as nvfp4_linear_fwd does (the same kernels in the
+ *     same order), bit for bit.  It skips the one step whose result only
+ *     nvfp4_linear_bwd reads (the X column copy for wgrad): there is no
+ *     allocation-free backward to read it.  X, W, Y as in nvfp4_linear_fwd.
+ *   - T, Cin, Cout: multiples of 64, each below 2^31 (NVFP4_ERR_SHAPE).
+ *   - Returns NVFP4_ERR_WORKSPACE, before enqueuing anything, when the part
+ *     of the linear workspace the forward uses (the scalars, the X row copy
+ *     and both W copies) exceeds the scratch size.
  *   - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
- *   - Its first call on a device looks up the scratch address on that device
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - The first call in each CUDA context looks up the scratch address in
+ *     that context (cudaGetSymbolAddress, cached by the context's id); make
+ *     that first call before any stream capture in the context.
  *   - Every call shares the one scratch area and leaves its contents behind
  *     (the quantized operands of the last call); each call rewrites what it
  *     reads.  Calls whose GPU work overlaps (other streams, other threads on

@@ -9,6 +9,7 @@
 #include "../../include/nvfp4.h"
 #include "common.cuh"
 #include "kernels.h"
+#include "linear.h"
 
 namespace {
 
@@ -100,14 +101,52 @@ nvfp4_tensor ws_tensor(void* ws, const WsLayout& L, int i) {
   return t;
 }
 
+// Shape rules of the linear layer: multiples of 64, each below 2^31 (the GEMM
+// limit), checked before any size arithmetic so ws_layout never overflows.
+bool linear_shape_ok(int64_t T, int64_t Cin, int64_t Cout) {
+  const int64_t lim = int64_t(1) << 31;
+  return T > 0 && Cin > 0 && Cout > 0 && T < lim && Cin < lim && Cout < lim && T % 64 == 0 && Cin % 64 == 0 &&
+         Cout % 64 == 0;
+}
+
 nvfp4_status linear_check(int64_t T, int64_t Cin, int64_t Cout, void* ws, size_t ws_bytes) {
-  if (T <= 0 || Cin <= 0 || Cout <= 0 || T % 64 || Cin % 64 || Cout % 64) return NVFP4_ERR_SHAPE;
+  if (!linear_shape_ok(T, Cin, Cout)) return NVFP4_ERR_SHAPE;
   if (!ws || ws_bytes < ws_layout(T, Cin, Cout).total) return NVFP4_ERR_WORKSPACE;
   if (!aligned16(ws)) return NVFP4_ERR_ALIGN;
   return NVFP4_OK;
 }
 
 }  // namespace
+
+namespace nvfp4 {
+
+size_t linear_forward_bytes(int64_t T, int64_t Cin, int64_t Cout) {
+  if (!linear_shape_ok(T, Cin, Cout)) return 0;
+  return ws_layout(T, Cin, Cout).data[3];   // tensors 0..2 and the scalars come first
+}
+
+nvfp4_status linear_forward(const void* X, const void* W, int64_t T, int64_t Cin, int64_t Cout, void* Y, void* ws,
+                            bool keep_wgrad, nvfp4_stream_t stream) {
+  const WsLayout L = ws_layout(T, Cin, Cout);
+  float* amax = static_cast<float*>(ws);
+  const nvfp4_tensor xr = ws_tensor(ws, L, 0), wr = ws_tensor(ws, L, 1), wc = ws_tensor(ws, L, 2);
+  nvfp4_status st;
+  // fprop operands: X row-wise (RN), W 2D (RN) with its transposed copy for dgrad
+  // one pass over X gives both its amax (row copy) and its RHT amax (column copy)
+  if ((st = nvfp4_amax(X, T, Cin, Cin, 2, amax + kAmaxX, stream)) != NVFP4_OK) return st;
+  if ((st = nvfp4_quantize(X, T, Cin, Cin, NVFP4_ROW, 0, 0, 0, amax + kAmaxX, &xr, nullptr, stream)) != NVFP4_OK)
+    return st;
+  if ((st = nvfp4_amax(W, Cout, Cin, Cin, 0, amax + kAmaxW, stream)) != NVFP4_OK) return st;
+  if ((st = nvfp4_quantize(W, Cout, Cin, Cin, NVFP4_2D, 0, 0, 0, amax + kAmaxW, &wr, &wc, stream)) != NVFP4_OK)
+    return st;
+  if ((st = nvfp4_gemm(&xr, &wr, Y, NVFP4_OUT_BF16, Cout, stream)) != NVFP4_OK) return st;
+  if (!keep_wgrad) return NVFP4_OK;
+  // wgrad operand saved for the backward pass: X^T with the RHT along tokens (RN)
+  const nvfp4_tensor xc = ws_tensor(ws, L, 3);
+  return nvfp4_quantize(X, T, Cin, Cin, NVFP4_COL, 1, 0, 0, amax + kAmaxXr, nullptr, &xc, stream);
+}
+
+}  // namespace nvfp4
 
 extern "C" {
 
@@ -295,14 +334,16 @@ nvfp4_status nvfp4_gemm_amax(const nvfp4_tensor* A, const nvfp4_tensor* B, void*
 }
 
 size_t nvfp4_linear_workspace_bytes(int64_t T, int64_t Cin, int64_t Cout) {
-  if (T <= 0 || Cin <= 0 || Cout <= 0) return 0;
+  const int64_t lim = int64_t(1) << 31;
+  if (T <= 0 || Cin <= 0 || Cout <= 0 || T >= lim || Cin >= lim || Cout >= lim) return 0;
   return ws_layout(T, Cin, Cout).total;
 }
 
 nvfp4_status nvfp4_linear_workspace_tensor(void* workspace, int64_t T, int64_t Cin, int64_t Cout, int which,
                                            nvfp4_tensor* out) {
   if (!workspace || !out || which < 0 || which >= kWsTensors) return NVFP4_ERR_INVALID_ARG;
-  if (T <= 0 || Cin <= 0 || Cout <= 0) return NVFP4_ERR_SHAPE;
+  const int64_t lim = int64_t(1) << 31;
+  if (T <= 0 || Cin <= 0 || Cout <= 0 || T >= lim || Cin >= lim || Cout >= lim) return NVFP4_ERR_SHAPE;
   *out = ws_tensor(workspace, ws_layout(T, Cin, Cout), which);
   return NVFP4_OK;
 }
@@ -313,21 +354,7 @@ nvfp4_status nvfp4_linear_fwd(const void* X, const void* W, int64_t T, int64_t C
   nvfp4_status st = linear_check(T, Cin, Cout, workspace, workspace_bytes);
   if (st != NVFP4_OK) return st;
   if (!aligned16(X) || !aligned16(W) || !aligned16(Y)) return NVFP4_ERR_ALIGN;
-  const WsLayout L = ws_layout(T, Cin, Cout);
-  float* amax = static_cast<float*>(workspace);
-  const nvfp4_tensor xr = ws_tensor(workspace, L, 0), wr = ws_tensor(workspace, L, 1),
-                     wc = ws_tensor(workspace, L, 2), xc = ws_tensor(workspace, L, 3);
-  // fprop operands: X row-wise (RN), W 2D (RN) with its transposed copy for dgrad
-  // one pass over X gives both its amax (row copy) and its RHT amax (column copy)
-  if ((st = nvfp4_amax(X, T, Cin, Cin, 2, amax + kAmaxX, stream)) != NVFP4_OK) return st;
-  if ((st = nvfp4_quantize(X, T, Cin, Cin, NVFP4_ROW, 0, 0, 0, amax + kAmaxX, &xr, nullptr, stream)) != NVFP4_OK)
-    return st;
-  if ((st = nvfp4_amax(W, Cout, Cin, Cin, 0, amax + kAmaxW, stream)) != NVFP4_OK) return st;
-  if ((st = nvfp4_quantize(W, Cout, Cin, Cin, NVFP4_2D, 0, 0, 0, amax + kAmaxW, &wr, &wc, stream)) != NVFP4_OK)
-    return st;
-  if ((st = nvfp4_gemm(&xr, &wr, Y, NVFP4_OUT_BF16, Cout, stream)) != NVFP4_OK) return st;
-  // wgrad operand saved for the backward pass: X^T with the RHT along tokens (RN)
-  return nvfp4_quantize(X, T, Cin, Cin, NVFP4_COL, 1, 0, 0, amax + kAmaxXr, nullptr, &xc, stream);
+  return nvfp4::linear_forward(X, W, T, Cin, Cout, Y, workspace, true, stream);
 }
 
 nvfp4_status nvfp4_linear_bwd(const void* dY, int64_t T, int64_t Cin, int64_t Cout, uint64_t seed, void* dX,
