@@ -9,6 +9,9 @@ FP64 GEMM); this module only marshals numpy arrays through ctypes.  The readings
 R1..R18 (NVFP4) and R21..R24 (the MXFP4 comparison format) that fix what the
 pages leave open are listed at the top of that file.
 
+Non-finite inputs follow reading R25 (NaN-propagating amax; a copy whose amax
+is not finite has all scales 0x7F, all codes 0).
+
 Parity unpinned: the storage layouts (R17 nibble order, R18 scale swizzle),
 the op-order readings (R4, R6, R9, R16) and the MXFP4 scale rule and clipping
 (R23, R24: the OCP Microscaling definition the pages name but do not spell
@@ -53,9 +56,9 @@ def lib():
             "orc_amax_rht": (ctypes.c_float, [_u16p, _i64, _i64, _i64]),
             "orc_global_scales": (None, [ctypes.c_float, _f32p]),
             "orc_quantize_row": (None, [_u16p, _i64, _i64, _i64, ctypes.c_float, ctypes.c_int,
-                                        ctypes.c_uint64, _u8p, _u8p]),
+                                        ctypes.c_uint64, _i64, _u8p, _u8p]),
             "orc_quantize_col": (None, [_u16p, _i64, _i64, _i64, ctypes.c_float, ctypes.c_int,
-                                        ctypes.c_int, ctypes.c_uint64, _u8p, _u8p]),
+                                        ctypes.c_int, ctypes.c_uint64, _i64, _u8p, _u8p]),
             "orc_quantize_2d": (None, [_u16p, _i64, _i64, _i64, ctypes.c_float, _u8p, _u8p]),
             "orc_pack_nibbles": (None, [_u8p, _i64, _i64, _u8p]),
             "orc_sf_offset": (_i64, [_i64, _i64, _i64]),
@@ -164,25 +167,28 @@ def global_scales(a):
     return out[0], out[1]
 
 
-def quantize_row(x, a, sr=False, seed=0):
-    """Row-wise 1x16.  Returns (codes [R, C] u8, sf [R, C/16] u8)."""
+def quantize_row(x, a, sr=False, seed=0, row0=0):
+    """Row-wise 1x16.  Returns (codes [R, C] u8, sf [R, C/16] u8).  row0: x is
+    rows row0.. of a larger tensor with C columns, whose element indices key the
+    SR draws (R12)."""
     x = _bf16_bits(x)
     R, C = x.shape
     codes = np.zeros((R, C), dtype=np.uint8)
     sf = np.zeros((R, C // 16), dtype=np.uint8)
-    lib().orc_quantize_row(_p(x, _u16p), R, C, C, float(a), int(bool(sr)), int(seed),
+    lib().orc_quantize_row(_p(x, _u16p), R, C, C, float(a), int(bool(sr)), int(seed), int(row0) * C,
                            _p(codes, _u8p), _p(sf, _u8p))
     return codes, sf
 
 
-def quantize_col(x, a, rht=False, sr=False, seed=0):
-    """Column-wise 1x16 along rows; transposed output (codes [C, R], sf [C, R/16])."""
+def quantize_col(x, a, rht=False, sr=False, seed=0, row0=0):
+    """Column-wise 1x16 along rows; transposed output (codes [C, R], sf [C, R/16]).
+    row0 as in quantize_row."""
     x = _bf16_bits(x)
     R, C = x.shape
     codes = np.zeros((C, R), dtype=np.uint8)
     sf = np.zeros((C, R // 16), dtype=np.uint8)
     lib().orc_quantize_col(_p(x, _u16p), R, C, C, float(a), int(bool(rht)), int(bool(sr)), int(seed),
-                           _p(codes, _u8p), _p(sf, _u8p))
+                           int(row0) * C, _p(codes, _u8p), _p(sf, _u8p))
     return codes, sf
 
 

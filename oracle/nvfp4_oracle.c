@@ -34,13 +34,22 @@
  *   R10 SR: round up iff (w >> 8) * 2^-24 < p, p the fractional position
  *   R11 Philox4x32-10, key = seed, counter = (idx>>2 lo, idx>>2 hi, domain, 0),
  *       word idx & 3
- *   R12 idx = r*C + c, the element's row-major index in the input [R, C]
+ *   R12 idx = r*C + c, the element's row-major index in the input [R, C]; for a
+ *       block of rows row0.. of a larger [*, C] tensor (one data-parallel
+ *       rank's token shard) idx = (row0 + r)*C + c, the index in the whole
+ *       tensor: the quantizers take idx0 = row0*C and add it
  *   R13 domain 0 = row-wise SR, 1 = column-wise SR, 2 = RHT signs
  *   R14 RHT signs: bit j of word 0 of Philox(key 0, counter (0,0,2,0)); set -> -1
  *   R15 the RHT acts on aligned 16-runs along the GEMM K dimension (tokens)
  *   R16 RHT FP32 order: signs, butterflies h = 1,2,4,8, then * 0.25
  *   R17 packing: element 2i in the low nibble, 2i+1 in the high nibble
  *   R18 scale layout: 128x4 tiles of 512 bytes (see orc_sf_offset)
+ *   R25 non-finite inputs: the amax of a tensor holding a NaN is NaN, of one
+ *       holding an infinity (and no NaN) +inf; the RHT amax of a tensor holding
+ *       any non-finite element is NaN.  A quantizer handed a non-finite amax
+ *       flags the copy instead of encoding it: every one of its block scales is
+ *       0x7F (the E4M3 NaN), every code 0, and s_g = A/2688 as in R4 (inf or
+ *       NaN), so any GEMM that reads the copy returns NaN.  Padding stays 0.
  * MXFP4, the format the pages compare NVFP4 against ("Pretraining Large Language
  * Models with NVFP4", section 2A: blocks of 32 instead of 16, UE8M0 instead of
  * E4M3 block scales; section 3: the 8B comparison), read as the OCP
@@ -240,22 +249,37 @@ static inline float bf16_to_f32(uint16_t b)
     return f;
 }
 
-/* max |x| over a row-major BF16 [R, C] tensor with row pitch ld (elements). */
+/* max |x| over a row-major BF16 [R, C] tensor with row pitch ld (elements);
+ * NaN if any element is NaN (R25). */
 float orc_amax(const uint16_t *x, int64_t R, int64_t C, int64_t ld)
 {
     float m = 0.0f;
-#pragma omp parallel for reduction(max : m) schedule(static)
+    int nan_seen = 0;
+#pragma omp parallel for reduction(max : m) reduction(|| : nan_seen) schedule(static)
     for (int64_t r = 0; r < R; r++)
         for (int64_t c = 0; c < C; c++) {
             float a = fabsf(bf16_to_f32(x[r * ld + c]));
-            if (a > m) m = a;
+            if (isnan(a)) nan_seen = 1;
+            else if (a > m) m = a;
         }
-    return m;
+    return nan_seen ? NAN : m;
 }
 
-/* max |Q x| where Q acts on each aligned 16-run of rows of every column (R15). */
+static int has_nonfinite(const uint16_t *x, int64_t R, int64_t C, int64_t ld)
+{
+    int bad = 0;
+#pragma omp parallel for reduction(|| : bad) schedule(static)
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t c = 0; c < C; c++)
+            if (!isfinite(bf16_to_f32(x[r * ld + c]))) bad = 1;
+    return bad;
+}
+
+/* max |Q x| where Q acts on each aligned 16-run of rows of every column (R15);
+ * NaN if the tensor holds a non-finite element (R25). */
 float orc_amax_rht(const uint16_t *x, int64_t R, int64_t C, int64_t ld)
 {
+    if (has_nonfinite(x, R, C, ld)) return NAN;
     float m = 0.0f;
 #pragma omp parallel for reduction(max : m) schedule(static)
     for (int64_t tb = 0; tb < R / 16; tb++)
@@ -305,14 +329,24 @@ static int quant_block(const float *v, int n, float s_enc, int sr, const uint32_
     return sf;
 }
 
+/* R25: a copy whose amax is not finite -- every scale 0x7F, every code 0. */
+static void flag_nonfinite(int64_t rows, int64_t cols, uint8_t *codes, uint8_t *sf, int64_t nsf)
+{
+    memset(codes, 0, (size_t)(rows * cols));
+    memset(sf, 0x7F, (size_t)nsf);
+}
+
 /* Row-wise 1x16 quantization (section 2B.3: activations and gradients).
- * codes: [R, C] one code per byte; sf: [R, C/16]. */
+ * codes: [R, C] one code per byte; sf: [R, C/16].  idx0: index of x[0][0] in
+ * the tensor whose row-major element index keys the SR draws (R12; 0 for a
+ * whole tensor, row0*C for rows row0.. of a larger one). */
 void orc_quantize_row(const uint16_t *x, int64_t R, int64_t C, int64_t ld, float amax, int sr,
-                      uint64_t seed, uint8_t *codes, uint8_t *sf)
+                      uint64_t seed, int64_t idx0, uint8_t *codes, uint8_t *sf)
 {
     float g[2];
-    orc_global_scales(amax, g);
     int64_t S = C / 16;
+    if (!isfinite(amax)) { flag_nonfinite(R, C, codes, sf, R * S); return; }
+    orc_global_scales(amax, g);
 #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < R; r++)
         for (int64_t b = 0; b < S; b++) {
@@ -321,7 +355,7 @@ void orc_quantize_row(const uint16_t *x, int64_t R, int64_t C, int64_t ld, float
             for (int i = 0; i < 16; i++) {
                 int64_t c = b * 16 + i;
                 v[i] = bf16_to_f32(x[r * ld + c]);
-                w[i] = sr ? orc_sr_word(seed, (uint64_t)(r * C + c), 0u) : 0u;
+                w[i] = sr ? orc_sr_word(seed, (uint64_t)(idx0 + r * C + c), 0u) : 0u;
             }
             sf[r * S + b] = (uint8_t)quant_block(v, 16, g[0], sr, w, codes + r * C + b * 16);
         }
@@ -330,13 +364,15 @@ void orc_quantize_row(const uint16_t *x, int64_t R, int64_t C, int64_t ld, float
 /* Column-wise 1x16 quantization along R (the GEMM K dimension of wgrad), with
  * an optional RHT on each 16-run and optional SR.  The output is the transposed
  * copy: codes_t [C, R], sf_t [C, R/16].  amax must be the amax of the tensor the
- * blocks are taken from (orc_amax_rht when rht is set). */
+ * blocks are taken from (orc_amax_rht when rht is set).  idx0 as in
+ * orc_quantize_row: element (r, c) draws the word of index idx0 + r*C + c. */
 void orc_quantize_col(const uint16_t *x, int64_t R, int64_t C, int64_t ld, float amax, int rht,
-                      int sr, uint64_t seed, uint8_t *codes_t, uint8_t *sf_t)
+                      int sr, uint64_t seed, int64_t idx0, uint8_t *codes_t, uint8_t *sf_t)
 {
     float g[2];
-    orc_global_scales(amax, g);
     int64_t S = R / 16;
+    if (!isfinite(amax)) { flag_nonfinite(C, R, codes_t, sf_t, C * S); return; }
+    orc_global_scales(amax, g);
 #pragma omp parallel for schedule(static)
     for (int64_t c = 0; c < C; c++)
         for (int64_t tb = 0; tb < S; tb++) {
@@ -346,7 +382,7 @@ void orc_quantize_col(const uint16_t *x, int64_t R, int64_t C, int64_t ld, float
             for (int i = 0; i < 16; i++) {
                 int64_t r = tb * 16 + i;
                 v[i] = bf16_to_f32(x[r * ld + c]);
-                w[i] = sr ? orc_sr_word(seed, (uint64_t)(r * C + c), 1u) : 0u;
+                w[i] = sr ? orc_sr_word(seed, (uint64_t)(idx0 + r * C + c), 1u) : 0u;
             }
             if (rht) orc_rht16_f32(v, y); else memcpy(y, v, sizeof y);
             sf_t[c * S + tb] = (uint8_t)quant_block(y, 16, g[0], sr, w, q);
@@ -360,8 +396,9 @@ void orc_quantize_2d(const uint16_t *w, int64_t N, int64_t K, int64_t ld, float 
                      uint8_t *codes, uint8_t *sf_tile)
 {
     float g[2];
-    orc_global_scales(amax, g);
     int64_t TN = N / 16, TK = K / 16;
+    if (!isfinite(amax)) { flag_nonfinite(N, K, codes, sf_tile, TN * TK); return; }
+    orc_global_scales(amax, g);
 #pragma omp parallel for schedule(static)
     for (int64_t bn = 0; bn < TN; bn++)
         for (int64_t bk = 0; bk < TK; bk++) {

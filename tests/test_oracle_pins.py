@@ -336,3 +336,77 @@ def test_gemm_integer_special_case_exact():
     ia = np.vectorize(lambda c: int(round(2 * val[int(c)])))(ca).astype(np.int64)
     ib = np.vectorize(lambda c: int(round(2 * val[int(c)])))(cb).astype(np.int64)
     assert np.array_equal(D * 4, (ia @ ib.T).astype(np.float64))
+
+
+def test_scale_offsets_match_documented_tile_layout():
+    rows = _rows("sf_layout.txt")
+    assert len(rows) >= 10
+    for r, c, sp, off in ([int(t) for t in row] for row in rows):
+        assert O.sf_offset(r, c, sp) == off, (r, c, sp)
+
+
+# ----------------------------------------------------------------- row blocks of a larger tensor (R12)
+@pytest.mark.parametrize("row0,rows", [(0, 32), (16, 48), (64, 16), (80, 48)])
+def test_row_block_quantize_equals_slice_of_whole_tensor(row0, rows):
+    # element (r, c) of a block that starts at row row0 draws the SR word of
+    # element (row0 + r, c) of the whole tensor, so quantizing the block with
+    # its row offset must reproduce the whole tensor's codes for those rows
+    x = synth.gradients(128, 96, 31)
+    a, ar = O.amax(x), O.amax_rht(x)
+    blk = x[row0:row0 + rows].contiguous()
+    whole_r = O.quantize_row(x, a, sr=True, seed=77)
+    part_r = O.quantize_row(blk, a, sr=True, seed=77, row0=row0)
+    assert np.array_equal(part_r[0], whole_r[0][row0:row0 + rows])
+    assert np.array_equal(part_r[1], whole_r[1][row0:row0 + rows])
+    whole_c = O.quantize_col(x, ar, rht=True, sr=True, seed=77)
+    part_c = O.quantize_col(blk, ar, rht=True, sr=True, seed=77, row0=row0)
+    assert np.array_equal(part_c[0], whole_c[0][:, row0:row0 + rows])
+    assert np.array_equal(part_c[1], whole_c[1][:, row0 // 16:(row0 + rows) // 16])
+    if row0:
+        # the offset matters: without it the block draws other words
+        assert not np.array_equal(O.quantize_row(blk, a, sr=True, seed=77)[0], part_r[0])
+
+
+def test_row_offset_reaches_the_counter_high_word():
+    # a block whose element indices / 4 pass 2^32: its words are those of the
+    # whole-tensor indices, read one by one from the generator
+    C, rows = 64, 16
+    row0 = (1 << 34) // C - 8            # the block straddles element index 2^34
+    x = synth.gradients(rows, C, 32)
+    a = O.amax(x)
+    codes, sf = O.quantize_row(x, a, sr=True, seed=5, row0=row0)
+    S_enc = float(O.global_scales(a)[0])
+    xf = x.float().numpy()
+    for r in (0, 7, 8, 15):
+        for b in range(C // 16):
+            blk = xf[r, b * 16:(b + 1) * 16]
+            sb = O.e4m3_decode(sf[r, b])
+            for i in range(16):
+                idx = (row0 + r) * C + b * 16 + i
+                y = np.float32(blk[i]) * (np.float32(S_enc) / np.float32(sb)) if sb else np.float32(0)
+                want = O.e2m1_encode_sr(float(y), O.sr_word(5, idx, 0)) if sb else 0
+                assert codes[r, b * 16 + i] == want, (r, b, i)
+
+
+# ----------------------------------------------------------------- non-finite inputs (R25)
+def test_amax_propagates_nan_and_inf_like_numpy():
+    x = synth.normal(48, 64, 33, std=2.0)
+    for planted in (float("inf"), float("-inf"), float("nan")):
+        y = x.clone()
+        y[17, 9] = planted
+        want = np.max(np.abs(y.float().numpy()))        # numpy's max propagates NaN
+        got = O.amax(y)
+        assert (math.isnan(got) and math.isnan(want)) or got == want, planted
+        assert math.isnan(O.amax_rht(y)), planted
+    assert O.amax(x) == np.max(np.abs(x.float().numpy()))
+
+
+@pytest.mark.parametrize("amax", [float("inf"), float("nan")])
+def test_nonfinite_amax_flags_every_copy(amax):
+    x = synth.normal(32, 64, 34)
+    for codes, sf in (O.quantize_row(x, amax), O.quantize_row(x, amax, sr=True, seed=3),
+                      O.quantize_col(x, amax, rht=True, sr=True, seed=3), O.quantize_2d(x, amax)):
+        assert not codes.any() and np.all(sf == 0x7F)
+        assert math.isnan(O.e4m3_decode(0x7F))
+    s_enc, s_g = O.global_scales(amax)
+    assert not math.isfinite(s_g)
