@@ -1,15 +1,23 @@
 """Benchmark of the NVFP4 quantized linear layer on B200.
 
-One step = one full pass of the hot path over one batch: forward (amax, X
-row quantize, W 2D quantize, fprop GEMM, X column quantize with RHT) and
-backward (dY amax, dY row quantize with SR, dgrad GEMM, dY RHT amax, dY column
-quantize with RHT + SR, wgrad GEMM), on the "full" workload: T = 16384 tokens,
-hidden 5120 -> FFN 20480 (a 12B hybrid Mamba-Transformer's FFN up-projection),
-seeded synthetic BF16 inputs resident in HBM.
+One step = one full pass of the hot path over one batch, through the
+data-parallel linear layer (nvfp4_bit_microscaled_b200.dp): forward (amax and
+RHT amax of X, X row quantize, W amax, W 2D quantize, fprop GEMM, X column
+quantize with RHT) and backward (amax and RHT amax of dY, dY row quantize with
+SR, dgrad GEMM, dY column quantize with RHT + SR, wgrad GEMM), with the
+all-reduces of the amaxes (MAX) and of dW (SUM) when there is more than one
+rank.  Inputs are seeded synthetic BF16 tensors resident in HBM.
+
+The headline workload is the largest configuration, "large outlier-heavy":
+T = 32768 tokens, 8192 -> 8192, X Student-t(3), W N(0, 0.02) with 0.01% of
+its entries x50, dY N(0, 1e-3); its three GEMMs are 32768x8192x8192,
+32768x8192x8192 and 8192x8192x32768.  The "full" workload (T = 16384,
+hidden 5120 -> FFN 20480, a 12B hybrid Mamba-Transformer's up-projection) is
+timed the same way and reported in its own object.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-Under torchrun (N > 1) every rank runs its own batch (weak scaling, no
-collective on the data path); rank 0 prints one JSON line.
+Under torchrun (N > 1) every rank holds T tokens of an N*T-token batch (weak
+scaling) and runs the data-parallel step over NCCL; rank 0 prints one JSON line.
 
 --impl reference times the CPU oracle (the plain C reference) on the host cores
 on a bounded sample of the same workload.
@@ -18,7 +26,6 @@ import argparse
 import hashlib
 import json
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -30,13 +37,24 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from nvfp4_bit_microscaled_b200 import api, synth  # noqa: E402
+from nvfp4_bit_microscaled_b200 import api, dp, synth  # noqa: E402
 
 METRIC = "NVFP4 GEMM TFLOPS (% dense FP4 peak); quantize GB/s (% HBM peak)"
-WORKLOAD = dict(name="full", T=16384, Cin=5120, Cout=20480, seed=2, sr_seed=2)
+WORKLOADS = {
+    "large": dict(name="large", T=32768, Cin=8192, Cout=8192, seed=3, sr_seed=3,
+                  desc="large outlier-heavy linear fwd+bwd: T=32768, Cin=8192, Cout=8192 (X Student-t(3), "
+                       "W N(0,0.02) with 0.01% entries x50, dY N(0,1e-3))"),
+    "full": dict(name="full", T=16384, Cin=5120, Cout=20480, seed=2, sr_seed=2,
+                 desc="full linear fwd+bwd: T=16384, Cin=5120, Cout=20480 (FFN up-projection of a 12B hybrid "
+                      "Mamba-Transformer; X N(0,1) with 0.1% outlier channels x100, W N(0,0.02), "
+                      "dY N(0,1e-3) x per-row lognormal)"),
+}
+HEADLINE = "large"
+WORKLOAD = WORKLOADS[HEADLINE]
 DENSE_FP4_DATASHEET_TFLOPS = 9000.0
 FP4_PER_BF16 = 4.0           # nominal dense FP4 : BF16 tensor ratio (9 : 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_PROFILE = os.path.join("profiles", "gemm_traffic.json")
 
 
 def load_peaks():
@@ -48,21 +66,26 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def gemm_traffic_from_profile():
-    """DRAM bytes per launch of the fprop GEMM from the committed ncu summary,
-    or None when the kernel source changed since the counters were taken."""
-    path = os.path.join(ROOT, "profiles", "gemm_nvf4_full.md")
+def fp4_peak(peaks, src):
+    """Dense FP4 roofline: 4 x the burst BF16 GEMM rate (the kernels are timed
+    in a sub-second region, where the part runs at its burst clock)."""
+    v = FP4_PER_BF16 * peaks["bf16_tflops"]
+    return v, f"{src}: 4 x bf16_tflops burst ({peaks['bf16_tflops']}) (nominal dense FP4:BF16 = 9:2.25)"
+
+
+def gemm_profile():
+    """The committed ncu figures of the headline fprop GEMM (DRAM bytes per
+    launch, tensor-pipe activity), or None when gemm.cu has changed since
+    they were taken (checked by the source hash stored with them)."""
+    path = os.path.join(ROOT, GEMM_PROFILE)
     if not os.path.exists(path):
         return None
-    text = open(path).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    h = re.search(r"gemm_source_sha256:\s*([0-9a-f]{64})", text)
-    if not m or not h:
-        return None
+    with open(path) as f:
+        prof = json.load(f)
     src = open(os.path.join(ROOT, "nvfp4_bit_microscaled_b200", "csrc", "gemm.cu"), "rb").read()
-    if hashlib.sha256(src).hexdigest() != h.group(1):
+    if hashlib.sha256(src).hexdigest() != prof.get("gemm_source_sha256"):
         return None
-    return float(m.group(1))
+    return prof
 
 
 class ClockSampler:
@@ -72,8 +95,9 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, enabled=True):
         self.gpu_index = gpu_index
+        self.enabled = enabled
         self.proc = None
         self.path = os.path.join(tempfile.gettempdir(), f"nvfp4_bench_clocks_{os.getpid()}_{gpu_index}.csv")
         self.t0 = self.t1 = None
@@ -85,6 +109,8 @@ class ClockSampler:
         self.t1 = time.time()
 
     def __enter__(self):
+        if not self.enabled:
+            return self
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
@@ -149,100 +175,90 @@ def max_over_ranks(value, device, world):
 
 
 # --------------------------------------------------------------------------- our arm
-class Step:
-    """The hot path as individual C-ABI calls, with CUDA events around each
-    kernel group so per-kernel durations are measured inside the timed region."""
+class EventTimer:
+    """timer(kind, fn) for DataParallelLinear: CUDA events around every call on
+    the current stream, so per-kernel durations come from inside the timed region."""
 
-    def __init__(self, X, W, dY, seed, record):
-        self.X, self.W, self.dY, self.seed = X, W, dY, seed
-        T, Cin = X.shape
-        Cout = W.shape[0]
-        dev = X.device
-        self.T, self.Cin, self.Cout = T, Cin, Cout
-        self.amax = torch.zeros(8, dtype=torch.float32, device=dev)
-        q = api.empty_qtensor
-        self.xr, self.wr, self.wc = q(T, Cin, dev), q(Cout, Cin, dev), q(Cin, Cout, dev)
-        self.xc, self.gr, self.gc = q(Cin, T, dev), q(T, Cout, dev), q(Cout, T, dev)
-        self.Y = torch.empty(T, Cout, dtype=torch.bfloat16, device=dev)
-        self.dX = torch.empty(T, Cin, dtype=torch.bfloat16, device=dev)
-        self.dW = torch.empty(Cout, Cin, dtype=torch.float32, device=dev)
-        self.record = record
+    def __init__(self):
+        self.record = False
         self.events = []          # (kind, start, end)
 
-    def _ev(self, kind, fn):
+    def __call__(self, kind, fn):
         if not self.record:
-            fn()
-            return
+            return fn()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
-        fn()
+        out = fn()
         e.record()
         self.events.append((kind, s, e))
+        return out
 
-    def __call__(self):
-        a = self.amax
-        X, W, dY = self.X, self.W, self.dY
-        # forward: one pass over X gives max|X| (row copy) and max|QX| (column copy)
-        self._ev("amax_both", lambda: api.amax(X, rht=2, out=a[0:2]))
-        self._ev("quant_row", lambda: api.quantize(X, api.ROW, a[0:1], row_out=self.xr))
-        self._ev("amax", lambda: api.amax(W, out=a[2:3]))
-        self._ev("quant_2d", lambda: api.quantize(W, api.TWO_D, a[2:3], row_out=self.wr, col_out=self.wc))
-        self._ev("gemm_fprop", lambda: api.gemm(self.xr, self.wr, api.OUT_BF16, out=self.Y))
-        self._ev("quant_col_rht", lambda: api.quantize(X, api.COL, a[1:2], rht=True, col_out=self.xc))
-        # backward
-        self._ev("amax_both", lambda: api.amax(dY, rht=2, out=a[3:5]))
-        self._ev("quant_row_sr", lambda: api.quantize(dY, api.ROW, a[3:4], sr=True, seed=self.seed, row_out=self.gr))
-        self._ev("gemm_dgrad", lambda: api.gemm(self.gr, self.wc, api.OUT_BF16, out=self.dX))
-        self._ev("quant_col_rht_sr", lambda: api.quantize(dY, api.COL, a[4:5], rht=True, sr=True, seed=self.seed,
-                                                          col_out=self.gc))
-        self._ev("gemm_wgrad", lambda: api.gemm(self.gc, self.xc, api.OUT_F32, out=self.dW))
 
-    KERNELS_PER_STEP = 11  # 3 amax + 5 quantize + 3 GEMM kernels (no scale padding at these shapes)
+KERNELS_PER_STEP = 11  # 3 amax + 5 quantize + 3 GEMM kernels (no scale padding at these shapes)
+QUANT_KINDS = ("quant_row", "quant_2d", "quant_col_rht", "quant_row_sr", "quant_col_rht_sr")
 
-    def flops(self):
-        return 3 * 2.0 * self.T * self.Cin * self.Cout
 
-    def kernel_bytes(self):
-        """Algorithmic HBM bytes per kernel kind (reads + writes of the data the op must touch)."""
-        T, Ci, Co = self.T, self.Cin, self.Cout
-        q = lambda r, c: r * c / 2 + r * c / 16          # packed codes + one scale byte per 16
-        return {
-            "amax": 2.0 * Ci * Co,
-            "amax_both": 2.0 * (T * Ci + T * Co),
-            "quant_row": 2.0 * T * Ci + q(T, Ci),
-            "quant_2d": 2.0 * Co * Ci + 2 * q(Co, Ci),
-            "quant_col_rht": 2.0 * T * Ci + q(T, Ci),
-            "quant_row_sr": 2.0 * T * Co + q(T, Co),
-            "quant_col_rht_sr": 2.0 * T * Co + q(T, Co),
-        }
+def kernel_bytes(T, Ci, Co):
+    """Algorithmic HBM bytes per step of each kernel kind (reads + writes of the data the op must touch)."""
+    q = lambda r, c: r * c / 2 + r * c / 16          # packed codes + one scale byte per 16
+    return {
+        "amax": 2.0 * Ci * Co,
+        "amax_both": 2.0 * (T * Ci + T * Co),
+        "quant_row": 2.0 * T * Ci + q(T, Ci),
+        "quant_2d": 2.0 * Co * Ci + 2 * q(Co, Ci),
+        "quant_col_rht": 2.0 * T * Ci + q(T, Ci),
+        "quant_row_sr": 2.0 * T * Co + q(T, Co),
+        "quant_col_rht_sr": 2.0 * T * Co + q(T, Co),
+    }
 
 
 def gemm_flops(T, Ci, Co):
     return {"gemm_fprop": 2.0 * T * Co * Ci, "gemm_dgrad": 2.0 * T * Ci * Co, "gemm_wgrad": 2.0 * Co * Ci * T}
 
 
-def run_ours(args, rank, world, device):
-    wl = WORKLOAD
+def make_inputs(wl, rank, device):
+    """This rank's T tokens of the batch (its own seed) and the replicated W."""
+    name, T, Ci, Co = wl["name"], wl["T"], wl["Cin"], wl["Cout"]
+    seed = wl["seed"] + 1000 * rank
+    if name == "large":
+        X = synth.heavy_activations(T, Ci, seed, device=device)
+        W = synth.weights(Co, Ci, wl["seed"], device=device, outlier_frac=1e-4, outlier_scale=50.0)
+        dY = synth.gradients(T, Co, seed, device=device, row_lognormal=False)
+    else:
+        X = synth.activations(T, Ci, seed, device=device)
+        W = synth.weights(Co, Ci, wl["seed"], device=device)
+        dY = synth.gradients(T, Co, seed, device=device)
+    return X, W, dY
+
+
+def time_step(wl, args, rank, world, device, clocks=True):
+    """W warm-up steps, then K timed steps of the data-parallel layer between
+    barriers; device time from CUDA events, max over ranks."""
     T, Ci, Co = wl["T"], wl["Cin"], wl["Cout"]
-    seed = wl["seed"] + 1000 * rank      # every rank owns its own batch
-    X = synth.activations(T, Ci, seed, device=device)
-    W = synth.weights(Co, Ci, wl["seed"], device=device)
-    dY = synth.gradients(T, Co, seed, device=device)
-    torch.cuda.synchronize()
-    step = Step(X, W, dY, wl["sr_seed"], record=False)
+    X, W, dY = make_inputs(wl, rank, device)
+    timer = EventTimer()
+    layer = dp.DataParallelLinear(T, Ci, Co, device, timer=timer)
+    Y = torch.empty(T, Co, dtype=torch.bfloat16, device=device)
+    dX = torch.empty(T, Ci, dtype=torch.bfloat16, device=device)
+    dW = torch.empty(Co, Ci, dtype=torch.float32, device=device)
+
+    def step():
+        layer.forward(X, W, Y=Y)
+        layer.backward(dY, wl["sr_seed"], dX=dX, dW=dW)
+
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     api.read_device_error(clear=True)
 
-    step.record = True
-    step.events = []
+    timer.record = True
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                      else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[torch.cuda.current_device()]) as clk:
+    phys = (torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+            else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[torch.cuda.current_device()])
+    with ClockSampler(phys, enabled=clocks) as clk:
         clk.mark_start()
         start.record()
         for _ in range(args.steps):
@@ -258,119 +274,152 @@ def run_ours(args, rank, world, device):
         raise RuntimeError(f"device error word {err} after the timed region")
 
     per_kind = {}
-    for kind, s, e in step.events:
+    for kind, s, e in timer.events:
         per_kind.setdefault(kind, []).append(s.elapsed_time(e))
-    # each kind runs a fixed number of times per step; average per launch
     avg_ms = {k: sum(v) / len(v) for k, v in per_kind.items()}
     total_ms = {k: sum(v) / args.steps for k, v in per_kind.items()}
-
-    ms_max = max_over_ranks(ms_total, device, world)
-    ms_step = ms_max / args.steps
-    flops_step = step.flops()
-    value = flops_step * world / (ms_step * 1e-3) / 1e12
+    ms_step = max_over_ranks(ms_total, device, world) / args.steps
+    flops_step = 3 * 2.0 * T * Ci * Co
 
     peaks, peak_src = load_peaks()
-    fp4_peak = FP4_PER_BF16 * peaks["bf16_tflops_sustained"]
-    gf = gemm_flops(T, Ci, Co)
-    g_ms = total_ms["gemm_fprop"] + total_ms["gemm_dgrad"] + total_ms["gemm_wgrad"]
-    gemm_tflops = {k: gf[k] / (avg_ms[k] * 1e-3) / 1e12 for k in gf}
-    fprop_achieved = gemm_tflops["gemm_fprop"]
-    kb = step.kernel_bytes()
-    q_kinds = ["quant_row", "quant_2d", "quant_col_rht", "quant_row_sr", "quant_col_rht_sr"]
-    q_bytes = sum(kb[k] for k in q_kinds)
-    q_ms = sum(total_ms[k] for k in q_kinds)
-    a_bytes = kb["amax"] + kb["amax_both"]
-    a_ms = total_ms["amax"] + total_ms["amax_both"]
+    fpeak, fpeak_src = fp4_peak(peaks, peak_src)
     hbm = peaks["hbm_gbs"]
-    traffic = gemm_traffic_from_profile()
-
+    gf = gemm_flops(T, Ci, Co)
+    kb = kernel_bytes(T, Ci, Co)
+    g_ms = sum(total_ms[k] for k in gf)
+    q_ms = sum(total_ms[k] for k in QUANT_KINDS)
+    a_ms = total_ms["amax"] + total_ms["amax_both"]
     kernels = {}
     for k in avg_ms:
-        entry = {"ms_per_launch": round(avg_ms[k], 4), "launches_per_step": len(per_kind[k]) // args.steps}
+        n = len(per_kind[k]) // args.steps
+        entry = {"ms_per_launch": round(avg_ms[k], 4), "launches_per_step": n}
         if k in gf:
             entry["tflops"] = round(gf[k] / (avg_ms[k] * 1e-3) / 1e12, 1)
-            entry["frac_fp4_peak"] = round(entry["tflops"] / fp4_peak, 4)
-        else:
-            nl = len(per_kind[k]) // args.steps
-            b = kb[k] / nl
-            entry["gbs"] = round(b / (avg_ms[k] * 1e-3) / 1e9, 1)
+            entry["frac_fp4_peak"] = round(entry["tflops"] / fpeak, 4)
+        elif k in kb:
+            entry["gbs"] = round(kb[k] / n / (avg_ms[k] * 1e-3) / 1e9, 1)
             entry["frac_hbm"] = round(entry["gbs"] / hbm, 4)
         kernels[k] = entry
-
-    result = {
-        "metric": METRIC,
-        "value": round(value, 2),
-        "unit": "TFLOP/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
+    return {
+        "workload": wl["desc"],
         "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, fp32 accumulate)",
-        "data": "synthetic (seeded; X ~ N(0,1) with 0.1% outlier channels x100, W ~ N(0,0.02), "
-                "dY ~ N(0,1e-3) x per-row lognormal)",
-        "config": workload_config(world),
+        "value": round(flops_step * world / (ms_step * 1e-3) / 1e12, 2),
         "gemm": {
             "tflops_gemm_only": round(sum(gf.values()) / (g_ms * 1e-3) / 1e12, 1),
-            "frac_fp4_peak": round(sum(gf.values()) / (g_ms * 1e-3) / 1e12 / fp4_peak, 4),
+            "frac_fp4_peak": round(sum(gf.values()) / (g_ms * 1e-3) / 1e12 / fpeak, 4),
             "frac_fp4_datasheet_9pf": round(sum(gf.values()) / (g_ms * 1e-3) / 1e12 / DENSE_FP4_DATASHEET_TFLOPS, 4),
             "share_of_step": round(g_ms / ms_step, 3),
         },
         "quantize": {
-            "gbs": round(q_bytes / (q_ms * 1e-3) / 1e9, 1),
-            "frac_hbm": round(q_bytes / (q_ms * 1e-3) / 1e9 / hbm, 4),
-            "amax_gbs": round(a_bytes / (a_ms * 1e-3) / 1e9, 1),
-            "amax_frac_hbm": round(a_bytes / (a_ms * 1e-3) / 1e9 / hbm, 4),
+            "gbs": round(sum(kb[k] for k in QUANT_KINDS) / (q_ms * 1e-3) / 1e9, 1),
+            "frac_hbm": round(sum(kb[k] for k in QUANT_KINDS) / (q_ms * 1e-3) / 1e9 / hbm, 4),
+            "amax_gbs": round((kb["amax"] + kb["amax_both"]) / (a_ms * 1e-3) / 1e9, 1),
+            "amax_frac_hbm": round((kb["amax"] + kb["amax_both"]) / (a_ms * 1e-3) / 1e9 / hbm, 4),
             "share_of_step": round((q_ms + a_ms) / ms_step, 3),
         },
         "kernels": kernels,
+        "_fprop": (gf["gemm_fprop"], avg_ms["gemm_fprop"], fpeak, fpeak_src),
+        "_clocks": clk.summary(),
+        "_tensors": (X, W, dY),
+    }
+
+
+def run_ours(args, rank, world, device):
+    wl = WORKLOAD
+    T, Ci, Co = wl["T"], wl["Cin"], wl["Cout"]
+    head = time_step(wl, args, rank, world, device)
+    flops, fprop_ms, fpeak, fpeak_src = head.pop("_fprop")
+    achieved = flops / (fprop_ms * 1e-3) / 1e12
+    prof = gemm_profile()
+    result = {
+        "metric": METRIC,
+        "value": head["value"],
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, fp32 accumulate)",
+        "data": "synthetic (seeded; X Student-t(3), W N(0,0.02) with 0.01% entries x50, dY N(0,1e-3))",
+        "config": workload_config(world),
+        "gemm": head["gemm"],
+        "quantize": head["quantize"],
+        "kernels": head["kernels"],
         "roofline": {
-            "kernel": "gemm_fp4_pair_kernel<false, false> (fprop, M=16384 N=20480 K=5120)",
+            "kernel": f"gemm_fp4_pair_kernel<false, false> (fprop, M={T} N={Co} K={Ci}, BF16 out)",
             "bound": "tensor",
-            "achieved": round(fprop_achieved, 1),
-            "peak": round(fp4_peak, 1),
+            "achieved": round(achieved, 1),
+            "peak": round(fpeak, 1),
             "unit": "TFLOP/s",
-            "frac": round(fprop_achieved / fp4_peak, 4),
-            "peak_source": f"{peak_src}: 4 x bf16_tflops_sustained ({peaks['bf16_tflops_sustained']}) "
-                           f"(nominal dense FP4:BF16 = 9:2.25)",
-            "frac_of_datasheet_9pf": round(fprop_achieved / DENSE_FP4_DATASHEET_TFLOPS, 4),
-            "traffic": traffic,
+            "frac": round(achieved / fpeak, 4),
+            "peak_source": fpeak_src,
+            "frac_of_datasheet_9pf": round(achieved / DENSE_FP4_DATASHEET_TFLOPS, 4),
+            "traffic": prof["traffic_bytes_per_launch"] if prof else None,
+            "tensor_pipe_pct": prof.get("tensor_pipe_pct") if prof else None,
             "algorithmic_bytes": (T + Co) * Ci * 0.5625 + T * Co * 2,
         },
-        "gpu_launches": Step.KERNELS_PER_STEP * args.steps,
-        "clocks": clk.summary(),
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": head["_clocks"],
     }
-    return result, (X, W, dY)
+    if world > 1:
+        result["nccl_ranks"] = torch.distributed.get_world_size()
+    tensors = head.pop("_tensors")
+    del tensors
+    torch.cuda.empty_cache()
+    other = dict(WORKLOADS["full"])
+    full = time_step(other, args, rank, world, device, clocks=False)
+    full.pop("_fprop"), full.pop("_clocks"), full.pop("_tensors")
+    result["full_workload"] = full
+    return result
 
 
-def run_e2e(args, rank, world, device, tensors):
-    """Same metric through the public linear_fwd/linear_bwd calls with host
-    buffers: every step copies its X, W, dY from pinned host memory to the
-    device and its Y, dX, dW back to pinned host memory, inside the timed
-    region.  Copies run on their own streams and are pipelined across steps
-    (inputs of step i+1 and outputs of step i-1 move while step i computes),
-    with two device buffer sets; the data dependencies are kept by events."""
-    X, W, dY = tensors
-    T, Ci = X.shape
-    Co = W.shape[0]
-    steps = max(2, min(args.steps, 32))   # enough that filling and draining the copy pipeline is a small part
+def run_e2e(args, rank, world, device):
+    """Same metric end to end through the public API with host buffers: every
+    step copies its X, W, dY from pinned host memory to the device and its Y,
+    dX, dW back to pinned host memory, inside the timed region.  One GPU runs
+    nvfp4_linear_fwd / nvfp4_linear_bwd (the C ABI's linear calls); several
+    run the data-parallel layer.  Copies run on their own streams and are
+    pipelined across steps (inputs of step i+1 and outputs of step i-1 move
+    while step i computes), with two device buffer sets; the data dependencies
+    are kept by events."""
+    wl = WORKLOAD
+    T, Ci, Co = wl["T"], wl["Cin"], wl["Cout"]
+    steps = max(2, min(args.steps, 24))   # enough that filling and draining the copy pipeline is a small part
+    X, W, dY = make_inputs(wl, rank, device)
     hin = [tuple(t.cpu().pin_memory() for t in (X, W, dY)) for _ in range(2)]
+    del X, W, dY
     hout = [(torch.empty(T, Co, dtype=torch.bfloat16).pin_memory(),
              torch.empty(T, Ci, dtype=torch.bfloat16).pin_memory(),
              torch.empty(Co, Ci, dtype=torch.float32).pin_memory()) for _ in range(2)]
-    din = [(torch.empty_like(X), torch.empty_like(W), torch.empty_like(dY)) for _ in range(2)]
-    dout = [(torch.empty(T, Co, dtype=torch.bfloat16, device=device), torch.empty(T, Ci, dtype=torch.bfloat16, device=device),
-             torch.empty(Co, Ci, dtype=torch.float32, device=device)) for _ in range(2)]
-    ws = [api.LinearWorkspace(T, Ci, Co, device) for _ in range(2)]
-    compute, h2d, d2h = torch.cuda.current_stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    din = [tuple(torch.empty_like(h, device=device) for h in hin[0]) for _ in range(2)]
+    dout = [tuple(torch.empty_like(h, device=device) for h in hout[0]) for _ in range(2)]
+    if world == 1:
+        ws = [api.LinearWorkspace(T, Ci, Co, device) for _ in range(2)]
+
+        def compute(b):
+            Xd, Wd, Gd = din[b]
+            Y, gX, gW = dout[b]
+            api.linear_fwd(Xd, Wd, ws[b], Y=Y)
+            api.linear_bwd(Gd, ws[b], wl["sr_seed"], dX=gX, dW=gW)
+    else:
+        layers = [dp.DataParallelLinear(T, Ci, Co, device) for _ in range(2)]
+
+        def compute(b):
+            Xd, Wd, Gd = din[b]
+            Y, gX, gW = dout[b]
+            layers[b].forward(Xd, Wd, Y=Y)
+            layers[b].backward(Gd, wl["sr_seed"], dX=gX, dW=gW)
+    compute_s, h2d, d2h = torch.cuda.current_stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
     def run(n):
         loaded = [None, None]      # event: inputs of buffer b on the device
         computed = [None, None]    # event: outputs of buffer b ready
         drained = [None, None]     # event: outputs of buffer b copied out (buffer b reusable)
         consumed = [None, None]    # event: inputs of buffer b no longer needed
+
         def load(i):
             b = i % 2
             with torch.cuda.stream(h2d):
@@ -385,37 +434,34 @@ def run_e2e(args, rank, world, device, tensors):
             b = i % 2
             if i + 1 < n:
                 load(i + 1)
-            compute.wait_event(loaded[b])
+            compute_s.wait_event(loaded[b])
             if drained[b] is not None:
-                compute.wait_event(drained[b])
-            Xd, Wd, Gd = din[b]
-            Y, gX, gW = dout[b]
-            api.linear_fwd(Xd, Wd, ws[b], Y=Y)
-            api.linear_bwd(Gd, ws[b], WORKLOAD["sr_seed"], dX=gX, dW=gW)
+                compute_s.wait_event(drained[b])
+            compute(b)
             consumed[b] = torch.cuda.Event()
-            consumed[b].record(compute)
+            consumed[b].record(compute_s)
             computed[b] = torch.cuda.Event()
-            computed[b].record(compute)
+            computed[b].record(compute_s)
             with torch.cuda.stream(d2h):
                 d2h.wait_event(computed[b])
                 for h, d in zip(hout[b], dout[b]):
                     h.copy_(d, non_blocking=True)
                 drained[b] = torch.cuda.Event()
                 drained[b].record(d2h)
-        compute.wait_event(drained[(n - 1) % 2])
+        compute_s.wait_event(drained[(n - 1) % 2])
         if n > 1:
-            compute.wait_event(drained[(n - 2) % 2])
+            compute_s.wait_event(drained[(n - 2) % 2])
 
     run(2)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(compute)
+    s.record(compute_s)
     h2d.wait_event(s)
     d2h.wait_event(s)
     run(steps)
-    e.record(compute)
+    e.record(compute_s)
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e), device, world)
     ms_step = ms / steps
@@ -424,15 +470,16 @@ def run_e2e(args, rank, world, device, tensors):
     d2h_b = sum(t.numel() * t.element_size() for t in hout[0])
     return {"value": round(flops * world / (ms_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b, "ms_per_step": round(ms_step, 3),
-            "steps": steps, "pipelined": "H2D of step i+1 and D2H of step i-1 overlap step i (copy streams)"}
+            "steps": steps, "api": "nvfp4_linear_fwd/_bwd" if world == 1 else "DataParallelLinear (NCCL)",
+            "pipelined": "H2D of step i+1 and D2H of step i-1 overlap step i (copy streams)"}
 
 
 # --------------------------------------------------------------------------- reference arm
 def oracle_sample(seconds_target=15.0):
-    """The CPU oracle on a bounded sample of the same workload: the six
+    """The CPU oracle on a bounded sample of the headline workload: the six
     quantizations of a 64-token slice of the batch and W's first 256 rows, and
-    FP64 GEMM entries sampled from the three GEMMs.  Returns (TFLOP/s of GEMM
-    work, cores, description)."""
+    FP64 GEMM entries sampled from fprop and wgrad.  Returns (TFLOP/s of GEMM
+    work, cores, description, seconds)."""
     import numpy as np
 
     import oracle as O
@@ -440,9 +487,9 @@ def oracle_sample(seconds_target=15.0):
     wl = WORKLOAD
     Ci, Co = wl["Cin"], wl["Cout"]
     Ts = 64
-    X = synth.activations(Ts, Ci, wl["seed"])
-    W = synth.weights(256, Ci, wl["seed"])
-    dY = synth.gradients(Ts, Co, wl["seed"])
+    X = synth.heavy_activations(Ts, Ci, wl["seed"])
+    W = synth.weights(256, Ci, wl["seed"], outlier_frac=1e-4, outlier_scale=50.0)
+    dY = synth.gradients(Ts, Co, wl["seed"], row_lognormal=False)
     rng = np.random.default_rng(0)
     flops = 0.0
     t0 = time.perf_counter()
@@ -466,19 +513,20 @@ def oracle_sample(seconds_target=15.0):
             break
     dt = time.perf_counter() - t0
     desc = (f"oracle (plain C, OpenMP) on host cores: amax/quantize of a {Ts}-token slice of X and dY and of "
-            f"W[:256], then FP64 GEMM entries sampled from fprop (K={Ci}) and wgrad (K={Ts}) for ~{seconds_target:.0f}s")
+            f"W[:256] of the large workload, then FP64 GEMM entries sampled from fprop (K={Ci}) and wgrad "
+            f"(K={Ts}) for ~{seconds_target:.0f}s")
     return flops / dt / 1e12, O.num_threads(), desc, dt
 
 
 def workload_config(world):
-    """The config object both arms print: the full linear layer's workload."""
+    """The config object both arms print: the headline workload."""
     T, Ci, Co = WORKLOAD["T"], WORKLOAD["Cin"], WORKLOAD["Cout"]
     return {
-        "workload": f"full linear fwd+bwd: T={T}, Cin={Ci}, Cout={Co} (FFN up-projection of a 12B hybrid "
-                    f"Mamba-Transformer); 3 GEMMs, 3 amax, 5 quantize kernels per step",
+        "workload": WORKLOAD["desc"] + "; 3 GEMMs, 3 amax, 5 quantize kernels per step",
         "T": T, "Cin": Ci, "Cout": Co,
-        "parallelism": f"independent batch per GPU x{world}",
-        "l2": "inputs larger than L2 (X 168 MB, W 210 MB, dY 671 MB; L2 126 MB): no flush needed",
+        "parallelism": f"dp{world}" + (" (NCCL all-reduce of amaxes and dW)" if world > 1 else ""),
+        "l2": f"inputs larger than L2 (X {2 * T * Ci / 1e6:.0f} MB, W {2 * Co * Ci / 1e6:.0f} MB, "
+              f"dY {2 * T * Co / 1e6:.0f} MB; L2 126 MB): no flush needed",
     }
 
 
@@ -544,13 +592,13 @@ def measure_mxfp4(X, W, reps=20):
     torch.cuda.synchronize()
     q_ms = _event_ms(lambda: api.mx_quantize(X, out=qx), reps)
     g_ms = _event_ms(lambda: api.mx_gemm(qx, qw, api.OUT_BF16, out=Y), reps)
-    peaks, _ = load_peaks()
-    fp4_peak = FP4_PER_BF16 * peaks["bf16_tflops_sustained"]
+    peaks, src = load_peaks()
+    fpeak, _ = fp4_peak(peaks, src)
     q_bytes = T * Ci * (2 + 0.5 + 1 / 32)
     tflops = 2.0 * T * Co * Ci / (g_ms * 1e-3) / 1e12
     gbs = q_bytes / (q_ms * 1e-3) / 1e9
     return {"gemm_fprop": {"ms_per_launch": round(g_ms, 4), "tflops": round(tflops, 1),
-                           "frac_fp4_peak": round(tflops / fp4_peak, 4)},
+                           "frac_fp4_peak": round(tflops / fpeak, 4)},
             "quant_row_x": {"ms_per_launch": round(q_ms, 4), "gbs": round(gbs, 1),
                             "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)},
             "note": "comparison format (1x32 blocks, UE8M0 scales, no tensor scale); not part of the step"}
@@ -722,12 +770,15 @@ def main():
     from nvfp4_bit_microscaled_b200 import build as libbuild
     libbuild.build()
 
-    result, tensors = run_ours(args, rank, world, device)
+    result = run_ours(args, rank, world, device)
     if not args.no_e2e:
-        result["e2e"] = run_e2e(args, rank, world, device, tensors)
-    result["mxfp4"] = measure_mxfp4(tensors[0], tensors[1])
-    result["epilogue_amax"] = measure_epilogue_amax(tensors[0], tensors[1])
-    del tensors
+        torch.cuda.empty_cache()
+        result["e2e"] = run_e2e(args, rank, world, device)
+    torch.cuda.empty_cache()
+    X, W, _ = make_inputs(WORKLOAD, rank, device)
+    result["mxfp4"] = measure_mxfp4(X, W)
+    result["epilogue_amax"] = measure_epilogue_amax(X, W)
+    del X, W
     if rank == 0 and not args.no_cpu_baseline:
         v, cores, desc, dt = oracle_sample(12.0)
         result["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}

@@ -12,7 +12,7 @@ import torch
 from . import _lib
 from ._lib import COL, OUT_BF16, OUT_F32, ROW, ROWCOL, TWO_D, Nvfp4Tensor, check, lib
 
-__all__ = ["QTensor", "empty_qtensor", "amax", "quantize", "gemm", "LinearWorkspace", "linear_fwd",
+__all__ = ["QTensor", "empty_qtensor", "amax", "quantize", "copy_is_flagged", "gemm", "LinearWorkspace", "linear_fwd",
            "linear_bwd", "read_device_error", "wait_probe", "rht_sign_mask", "data_bytes", "scale_bytes",
            "ROW", "COL", "ROWCOL", "TWO_D", "OUT_F32", "OUT_BF16"]
 
@@ -92,6 +92,14 @@ def quantize(x, mode, amax_dev, rht=False, sr=False, seed=0, row_out=None, col_o
                                   ctypes.byref(cd) if cd else None, _stream(x.device))
         check("nvfp4_quantize", st)
     return (row_out if want_row else None), (col_out if want_col else None)
+
+
+def copy_is_flagged(q):
+    """Host-side check of a quantized copy: True when its per-tensor amax was
+    not finite (a NaN or an infinity in the tensor), in which case the kernels
+    wrote 0x7F (the E4M3 NaN) to every block scale, 0 to every code, and a
+    non-finite decode scale.  Reads one float back (synchronizes the stream)."""
+    return not torch.isfinite(q.global_scale).all().item()
 
 
 def gemm(A, B, out_dtype=OUT_F32, out=None):

@@ -75,6 +75,11 @@ __global__ void __launch_bounds__(256) amax_rows_kernel(const uint16_t* __restri
 // after the maximum (an exact power-of-two scale commutes with max), and the
 // transform's last butterfly stage is folded into the maximum
 // (fwht16_absmax).
+// Non-finite inputs: every thread also keeps the BF16 magnitude maximum of
+// what it read; a NaN or infinity there (bits >= 0x7F80) makes its RHT
+// maximum NaN, and the reduction runs on float bit patterns, where the NaN
+// 0x7FC00000 orders above every finite value and infinity, so the result is
+// NaN exactly when the tensor holds a non-finite element.
 template <bool BOTH>
 __global__ void __launch_bounds__(256, 3) amax_rht_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
                                                             int64_t ld, unsigned int* __restrict__ out) {
@@ -96,11 +101,9 @@ __global__ void __launch_bounds__(256, 3) amax_rht_kernel(const uint16_t* __rest
     uint2 v[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __ldcs(reinterpret_cast<const uint2*>(base + i * ld));
-    if (BOTH) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        mplain = __vmaxu2(mplain, __vmaxu2(v[i].x & 0x7FFF7FFFu, v[i].y & 0x7FFF7FFFu));
-    }
+    for (int i = 0; i < 16; ++i)
+      mplain = __vmaxu2(mplain, __vmaxu2(v[i].x & 0x7FFF7FFFu, v[i].y & 0x7FFF7FFFu));
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       float f[16];
@@ -113,15 +116,12 @@ __global__ void __launch_bounds__(256, 3) amax_rht_kernel(const uint16_t* __rest
       m = fmaxf(m, fwht16_absmax<false>(f));
     }
   }
-  m = __fmul_rn(m, 0.25f);
   uint32_t mp = max(mplain & 0xFFFFu, mplain >> 16);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    if (BOTH) mp = max(mp, __shfl_xor_sync(0xFFFFFFFFu, mp, o));
-  }
+  uint32_t mb = mp >= 0x7F80u ? 0x7FC00000u : __float_as_uint(__fmul_rn(m, 0.25f));
+  mb = __reduce_max_sync(0xFFFFFFFFu, mb);
+  if (BOTH) mp = __reduce_max_sync(0xFFFFFFFFu, mp);
   if ((threadIdx.x & 31) == 0) {
-    if (m > 0.0f) atomicMax(out + (BOTH ? 1 : 0), __float_as_uint(m));
+    if (mb) atomicMax(out + (BOTH ? 1 : 0), mb);
     if (BOTH && mp) atomicMax(out, mp << 16);
   }
 }

@@ -205,30 +205,34 @@ __device__ __forceinline__ u32x4 sr_words(uint64_t g, uint32_t domain, uint32_t 
 // ("Pretraining Large Language Models with NVFP4", section 2B.4 and the
 // "De Gok" example: 3.4 goes to 4 with probability 0.4.)
 //
-// On [1, 6] the E2M1 grid is the FP32 values with one mantissa bit, so p is
+// |y| >= 1: the E2M1 grid is the FP32 values with one mantissa bit, so p is
 // the 22 bits below it over 2^22, and u < p  <=>  (w >> 10) < frac22  <=>
-// frac22 + ((~w) >> 10) carries into that bit: add and truncate.  On [0.5, 1)
-// the grid is {0.5, 1} and the same holds with 23 bits and (~w) >> 9.  Below
-// 0.5 (grid {0, 0.5}, p = 2a) the comparison (w >> 8) < a * 2^25 is done in
-// FP32 (both sides exact).  Every case is the same decision as the
-// definition above, bit for bit.
+// frac22 + ((~w) >> 10) carries into that bit: add and truncate, on the
+// signed bit pattern (the carry never reaches the sign bit and the mask keeps
+// it).  (~w) >> 10 == (2^22 - 1) - (w >> 10): one three-input add.  It also
+// runs without the saturation at 6: a value in (6, 6.4] (the E4M3 block scale
+// rounds to nearest, so |y| stays below 6.4) comes out as 6 or 8, and the
+// saturating E2M1 conversion turns both into 6, the code the saturated value
+// gives.
 //
-// The add-and-truncate runs on the signed bit pattern (the carry never reaches
-// the sign bit, and the mask keeps it), and without the saturation at 6: a
-// value in (6, 6.4] (the E4M3 block scale rounds to nearest, so |y| stays
-// below 6.4) comes out as 6 or 8, and the saturating E2M1 conversion turns
-// both into 6, the code the saturated value gives.
+// |y| < 1: the grid is {0, 0.5, 1}, a lattice of step 0.5, and the rule is
+// q = ceil_0.5(|y| - u/2) exactly (round up iff p > u).  It is evaluated in
+// FP32 with upward rounding: z = RU(|y| - 2^-25 (w >> 8)) is one fma, and
+// ceil_0.5(RU(x)) = ceil_0.5(x) for every real x because the lattice points
+// are floats; RU(z + 1.5 * 2^22) - 1.5 * 2^22 then takes the ceiling on the
+// lattice (z + 1.5 * 2^22 lies in a binade whose ulp is 0.5).  Exact for every
+// |y| < 1, tiny values included, with no integer work: the rounding runs on
+// the FMA pipe, which these kernels leave idle, instead of the integer ALU
+// pipe they are bound by.
+//
+// Both are the same decision as the definition above, bit for bit.
 __device__ __forceinline__ float sr_magnitude(float y, uint32_t w) {
-  const float a = fabsf(y);
   const uint32_t b = __float_as_uint(y);
-  const bool big = a >= 1.0f;
-  // (~w) >> sh == (2^(32-sh) - 1) - (w >> sh) == low - (w >> sh), with low
-  // the bits below the kept ones: one three-input add, no bitwise not
-  const uint32_t low = big ? 0x003FFFFFu : 0x007FFFFFu;
-  const float upper = __uint_as_float((b + low - (w >> (big ? 10 : 9))) & ~low);
-  // below 0.5: (w >> 8) < a * 2^25 (exact) <=> (w >> 8) < ceil(a * 2^25), an integer below 2^24
-  const float lower = ((w >> 8) < __float2uint_ru(__fmul_rn(a, 33554432.0f))) ? 0.5f : 0.0f;  // 2^25
-  return a >= 0.5f ? upper : copysignf(lower, y);
+  const float upper = __uint_as_float((b + 0x003FFFFFu - (w >> 10)) & ~0x003FFFFFu);
+  const float z = __fmaf_ru(-2.98023223876953125e-08f, __uint2float_rn(w >> 8), fabsf(y));  // -2^-25
+  const float q = __fsub_rn(__fadd_ru(z, 6291456.0f), 6291456.0f);                            // 1.5 * 2^22
+  const float lower = __uint_as_float(__float_as_uint(q) | (b & 0x80000000u));
+  return fabsf(y) >= 1.0f ? upper : lower;
 }
 
 // --------------------------------------------------------------------------

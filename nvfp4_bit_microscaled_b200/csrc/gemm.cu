@@ -383,7 +383,16 @@ constexpr uint32_t P_OFF_BAR = P_OFF_STG + NUM_EPI_WARPS * P_STG_BYTES;
 constexpr uint32_t P_SMEM_BYTES = P_OFF_BAR + 512 + 1024;
 static_assert(P_OFF_STG % 1024 == 0, "swizzled staging boxes need 1024-byte alignment");
 static_assert(P_SMEM_BYTES <= 232448, "pair kernel shared memory exceeds the per-block limit");
-constexpr int P_GROUP_M = 8;
+
+// Tile raster of the pair kernel: groups of group_m consecutive M-tiles walk
+// the N-tiles together (M fastest), so each B tile is read from DRAM once per
+// group while the group's A tiles stay in L2.  The launcher sizes group_m.
+__device__ __forceinline__ void pair_tile(int t, int num_m, int num_n, int group_m, int* tm, int* tn) {
+  const int per_group = group_m * num_n, grp = t / per_group, first_m = grp * group_m;
+  const int gsize = min(num_m - first_m, group_m), within = t - grp * per_group;
+  *tm = first_m + within % gsize;
+  *tn = within / gsize;
+}
 
 // kind::mxf4nvf4 (NVFP4: UE4M3 scales) or kind::mxf4 (MXFP4: UE8M0 scales,
 // bit 23), A/B E2M1 K-major, M = 256 (pair), N = 256.
@@ -417,7 +426,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmD, const uint8_t* __restrict__ sfa,
                       const uint8_t* __restrict__ sfb, const float* __restrict__ gsa,
-                      const float* __restrict__ gsb, int M, int N, int K, int out_bf16,
+                      const float* __restrict__ gsb, int M, int N, int K, int out_bf16, int group_m,
                       float* __restrict__ amax_out) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -479,9 +488,8 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     bool issued[P_STAGES];
     for (int s = 0; s < P_STAGES; ++s) issued[s] = false, issued_parity[s] = 0;
     for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
-      const int per_group = P_GROUP_M * num_n, grp = t / per_group, first_m = grp * P_GROUP_M;
-      const int gsize = min(num_m - first_m, P_GROUP_M), within = t - grp * per_group;
-      const int tm = first_m + within % gsize, tn = within / gsize;
+      int tm, tn;
+      pair_tile(t, num_m, num_n, group_m, &tm, &tn);
       for (int kt = 0; kt < num_kt; ++kt) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, kErrWaitEmpty)) { *abort_flag = 1; break; }
         const int nkb = min(KB_PER_STAGE, katoms - kt * KB_PER_STAGE);
@@ -563,9 +571,8 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     int stage = 0;
     uint32_t phase = 0;
     for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
-      const int per_group = P_GROUP_M * num_n, grp = t / per_group, first_m = grp * P_GROUP_M;
-      const int gsize = min(num_m - first_m, P_GROUP_M), within = t - grp * per_group;
-      const int tm = first_m + within % gsize, tn = within / gsize;
+      int tm, tn;
+      pair_tile(t, num_m, num_n, group_m, &tm, &tn);
       // scale blocks past the padded scale matrix were not loaded: zeros instead
       const bool a_sf = 2 * tm + static_cast<int>(rank) < sf_rows_a;
       const bool b_sf0 = 2 * tn < sf_rows_b, b_sf1 = 2 * tn + 1 < sf_rows_b;
@@ -622,9 +629,8 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     uint32_t acc_phase = 0;
     float run_max = 0.0f;  // AMAX only
     for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
-      const int per_group = P_GROUP_M * num_n, grp = t / per_group, first_m = grp * P_GROUP_M;
-      const int gsize = min(num_m - first_m, P_GROUP_M), within = t - grp * per_group;
-      const int tm = first_m + within % gsize, tn = within / gsize;
+      int tm, tn;
+      pair_tile(t, num_m, num_n, group_m, &tm, &tn);
       if (!mbar_wait_cluster(acc_full, acc_phase, kErrWaitAccFull)) { *abort_flag = 1; break; }
       tc_fence_after();
       const int row0 = tm * 256 + 128 * static_cast<int>(rank) + quarter * 32;
@@ -723,35 +729,66 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
+// Encoded tensor maps, cached by every input of the encoding (address, shape,
+// pitch, box, element type), so a hit returns the map the encoder would
+// produce again: a repeated GEMM on the same buffers skips the three driver
+// encode calls.  A small direct-mapped table; a miss overwrites its slot.
+struct MapKey {
+  uintptr_t addr;
+  int64_t dim0, dim1, pitch;
+  int box0, box1, kind;   // kind: 0 packed operand, 1 BF16 output, 2 FP32 output
+  bool operator==(const MapKey& o) const {
+    return addr == o.addr && dim0 == o.dim0 && dim1 == o.dim1 && pitch == o.pitch && box0 == o.box0 &&
+           box1 == o.box1 && kind == o.kind;
+  }
+};
+
+bool cached_encode(const MapKey& key, CUtensorMap* tm, CUtensorMapDataType dtype, CUtensorMapL2promotion l2) {
+  constexpr int kSlots = 64;
+  static std::mutex mu;
+  static MapKey keys[kSlots];
+  static CUtensorMap maps[kSlots];
+  static bool used[kSlots] = {};
+  const size_t h = (key.addr >> 8) ^ static_cast<size_t>(key.dim0 * 31 + key.dim1 * 17 + key.kind * 7 + key.box1);
+  const int slot = static_cast<int>(h % kSlots);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (used[slot] && keys[slot] == key) {
+      *tm = maps[slot];
+      return true;
+    }
+  }
+  auto encode = get_encode_fn();
+  if (!encode) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(key.dim0), static_cast<cuuint64_t>(key.dim1)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(key.pitch)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(key.box0), static_cast<cuuint32_t>(key.box1)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(tm, dtype, 2, reinterpret_cast<void*>(key.addr), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  keys[slot] = key;
+  maps[slot] = *tm;
+  used[slot] = true;
+  return true;
+}
+
 // K-major packed FP4 operand [rows, K/2] bytes; box = 128 bytes x box_rows,
 // 128-byte swizzle (the canonical K-major layout the MMA descriptors name).
 bool make_operand_map(CUtensorMap* tm, const void* data, int64_t rows, int64_t K, int box_rows) {
-  auto encode = get_encode_fn();
-  if (!encode) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK_BYTES), static_cast<cuuint32_t>(box_rows)};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(data), dims, strides, box, estr,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  const MapKey key{reinterpret_cast<uintptr_t>(data), K / 2, rows, K / 2, BK_BYTES, box_rows, 0};
+  return cached_encode(key, tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
 // Output D [M, N] (row stride ldd elements), stored in 32-row x 128-byte boxes
 // (64 BF16 or 32 FP32 columns) from 128-byte-swizzled shared memory.
 bool make_output_map(CUtensorMap* tm, void* D, int64_t M, int64_t N, int64_t ldd, int out_bf16) {
-  auto encode = get_encode_fn();
-  if (!encode) return false;
   const int64_t esize = out_bf16 ? 2 : 4;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldd * esize)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 32};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode(tm, out_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, D, dims,
-                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                      CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  const MapKey key{reinterpret_cast<uintptr_t>(D), N, M, ldd * esize, static_cast<int>(128 / esize), 32,
+                   out_bf16 ? 1 : 2};
+  return cached_encode(key, tm, out_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                       CU_TENSOR_MAP_L2_PROMOTION_NONE);
 }
 
 // Per-device, per-kernel launch setup, done once: the dynamic shared-memory
@@ -834,6 +871,13 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
     if (e != cudaSuccess) return e;
     const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const int pairs = static_cast<int>(tiles < mp ? tiles : mp);
+    // Raster group: as many M-tiles as keep their A tiles (256 rows of packed
+    // codes and scales) within 48 MiB of the 126 MB L2, so that B tiles are
+    // re-read from DRAM once per group and the group's A tiles are not.
+    const int64_t num_m = (M + 255) / 256;
+    const int64_t a_tile_bytes = 256 * (K / 2 + (mx ? K / 32 : K / 16));
+    int64_t group_m = (int64_t(48) << 20) / a_tile_bytes;
+    group_m = group_m < 1 ? 1 : (group_m > num_m ? num_m : group_m);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
     cfg.blockDim = dim3(NUM_THREADS);
@@ -847,7 +891,8 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmD, sa, sb, a_gs, b_gs, static_cast<int>(M),
-                              static_cast<int>(N), static_cast<int>(K), out_bf16, amax_out);
+                              static_cast<int>(N), static_cast<int>(K), out_bf16, static_cast<int>(group_m),
+                              amax_out);
   }
   auto kern = amax_out ? gemm_nvf4_kernel<true> : gemm_nvf4_kernel<false>;
   cudaError_t e =

@@ -26,6 +26,22 @@ __device__ __forceinline__ uint32_t pack8(const float* y) {
   return clear_negative_zero(f32x8_to_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]));
 }
 
+// A copy whose per-tensor amax is not finite (a NaN or an infinity in the
+// tensor) is flagged instead of encoded: every block scale of its rows x S
+// blocks is 0x7F (the E4M3 NaN) and every code is 0, so a GEMM that reads it
+// returns NaN.  Padding bytes are left to the padding kernel (zeros).  Runs
+// only on that path: the kernels branch here, uniformly, before any work.
+__device__ __noinline__ void flag_copy(uint8_t* __restrict__ data, int64_t rows, int64_t row_bytes,
+                                       uint8_t* __restrict__ sf, int64_t S, int64_t sp) {
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nt = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = t0; i < rows * row_bytes; i += nt) data[i] = 0;
+  for (int64_t i = t0; i < rows * S; i += nt) {
+    const int64_t r = i / S, c = i - r * S;
+    sf[sf_offset(r, c, sp)] = 0x7F;
+  }
+}
+
 __device__ __forceinline__ void unpack8(uint4 v, float* f) {
   f[0] = bf16_bits_to_f32(v.x & 0xFFFFu); f[1] = bf16_bits_to_f32(v.x >> 16);
   f[2] = bf16_bits_to_f32(v.y & 0xFFFFu); f[3] = bf16_bits_to_f32(v.y >> 16);
@@ -52,6 +68,10 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
   const float amax = __ldg(amax_dev);
   const float s_enc = encode_scale(amax);
   if (blockIdx.x == 0 && threadIdx.x == 0 && gs_out) *gs_out = decode_scale(amax);
+  if (!isfinite(amax)) {
+    flag_copy(data, R, C >> 1, sf, C >> 4, sp);
+    return;
+  }
   fill_r_table(r_tbl, s_enc);
   __syncthreads();
   const int lane = threadIdx.x & 31;
@@ -146,6 +166,10 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
   const float amax = __ldg(amax_dev);
   const float s_enc = encode_scale(amax);
   if (blockIdx.x == 0 && threadIdx.x == 0 && gs_out) *gs_out = decode_scale(amax);
+  if (!isfinite(amax)) {
+    flag_copy(data, C, R >> 1, sf, R >> 4, sp);
+    return;
+  }
   fill_r_table(r_tbl, s_enc);
   __syncthreads();
   const int64_t S = R >> 4;
@@ -232,6 +256,97 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
 }
 
 // ---------------------------------------------------------------------------
+// Column-wise 1x16 with round-to-nearest (the RHT copy of X for wgrad, and the
+// plain column copy): the same item, layout and arithmetic as quant_col_kernel
+// without SR, restructured for memory-level parallelism.  These copies are
+// bound by load latency, not by any pipe: the kernel above issues a block's
+// sixteen row loads only after it finished the previous block.  Here the
+// sixteen 8-byte loads of block b + 1 are issued before block b is computed
+// (two register buffers), and a block's four channels are unpacked and
+// processed one at a time, which keeps that second buffer within the
+// register budget of two CTAs per SM.
+// ---------------------------------------------------------------------------
+template <bool RHT>
+__global__ void __launch_bounds__(256, 2) quant_col_rn_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+                                                                int64_t ld, const float* __restrict__ amax_dev,
+                                                                uint8_t* __restrict__ data, uint8_t* __restrict__ sf,
+                                                                int64_t sp, float* __restrict__ gs_out) {
+  __shared__ float r_tbl[kRTableSize];
+  const float amax = __ldg(amax_dev);
+  const float s_enc = encode_scale(amax);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && gs_out) *gs_out = decode_scale(amax);
+  if (!isfinite(amax)) {
+    flag_copy(data, C, R >> 1, sf, R >> 4, sp);
+    return;
+  }
+  fill_r_table(r_tbl, s_enc);
+  __syncthreads();
+  const int64_t S = R >> 4;
+  const int64_t nq = (S + 3) >> 2;
+  const int64_t ng = C >> 2;
+  const int64_t items = nq * ng;
+  const int64_t half_r = R >> 1;
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x, step_q = step / ng, step_r = step - step_q * ng;
+  int64_t q_next = first / ng, g_next = first - q_next * ng;
+
+  for (int64_t it = first; it < items; it += step) {
+    const int64_t q = q_next, g = g_next;
+    g_next += step_r;
+    q_next += step_q;
+    if (g_next >= ng) g_next -= ng, ++q_next;
+    const int64_t c0 = g * 4, t0 = q * 64;
+    const int nb = static_cast<int>((S - 4 * q) < 4 ? (S - 4 * q) : 4);
+    const uint16_t* src = x + t0 * ld + c0;
+    uint32_t sfw[4] = {0u, 0u, 0u, 0u};
+    // block tb of the item -> codes of its four channels, scale bytes into sfw
+    auto block = [&](const uint2 (&cur)[16], int tb) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {   // one channel at a time: 16 floats live
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t w = (c < 2) ? cur[i].x : cur[i].y;
+          v[i] = __uint_as_float((c & 1) ? (w & 0xFFFF0000u) : (w << 16));
+          if (RHT && rht_negates(i)) v[i] = -v[i];  // s_i x_i
+        }
+        float m = 0.0f;
+        if (RHT) {
+          m = __fmul_rn(fwht16_absmax<true>(v), 0.25f);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.25f);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+        }
+        const BlockScale bs = block_scale_t(m, s_enc, r_tbl);
+        sfw[c] |= bs.sf << (8 * tb);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], bs.r);
+        reinterpret_cast<uint2*>(data + (c0 + c) * half_r + t0 / 2)[tb] = make_uint2(pack8(v), pack8(v + 8));
+      }
+    };
+    auto load = [&](uint2 (&dst)[16], int tb) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) dst[i] = __ldcs(reinterpret_cast<const uint2*>(src + (16 * tb + i) * ld));
+    };
+    uint2 bufa[16], bufb[16];
+    load(bufa, 0);
+#pragma unroll 1
+    for (int tb = 0; tb < nb; tb += 2) {   // blocks tb (bufa) and tb + 1 (bufb), each loaded one block ahead
+      if (tb + 1 < nb) load(bufb, tb + 1);
+      block(bufa, tb);
+      if (tb + 1 < nb) {
+        if (tb + 2 < nb) load(bufa, tb + 2);
+        block(bufb, tb + 1);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) *reinterpret_cast<uint32_t*>(sf + sf_offset(c0 + c, 4 * q, sp)) = sfw[c];
+  }
+}
+
+// ---------------------------------------------------------------------------
 // 2D 16x16 (weights).  CTA slab: 64 rows (4 tile rows) x 128 columns (8 tile
 // columns) of W.  Warp w takes tile row w/2 and tile columns 4*(w%2) .. +3;
 // eight lanes share a tile, lane l holding columns 2*(l%8), +1 of tile l/8
@@ -257,6 +372,11 @@ __global__ void __launch_bounds__(256, 4) quant_2d_kernel(const uint16_t* __rest
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     if (row_gs) *row_gs = decode_scale(amax);
     if (col_gs) *col_gs = decode_scale(amax);
+  }
+  if (!isfinite(amax)) {
+    if (row_data) flag_copy(row_data, N, K >> 1, row_sf, K >> 4, row_sp);
+    if (col_data) flag_copy(col_data, K, N >> 1, col_sf, N >> 4, col_sp);
+    return;
   }
   fill_r_table(r_tbl, s_enc);
   __syncthreads();
@@ -497,13 +617,13 @@ cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, co
   else if (rht && sr)
     quant_col_kernel<true, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else if (rht)
-    quant_col_kernel<true, false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
+    quant_col_rn_kernel<true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, d, f, sp, gs_out);
   else if (sr && narrow)
     quant_col_kernel<false, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else if (sr)
     quant_col_kernel<false, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else
-    quant_col_kernel<false, false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
+    quant_col_rn_kernel<false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, d, f, sp, gs_out);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_sf_pad_zero(scales, C, S, s);

@@ -7,7 +7,9 @@ path ("Pretraining Large Language Models with NVFP4", sections 2A and 2B):
 - the per-tensor scale of X, Q.X, dY and Q.dY comes from the amax of the
   whole batch (two-level scaling), so each pass all-reduces (MAX) its local
   amaxes, two floats in one collective, before any quantize kernel runs;
-- the partial FP32 weight gradients of the ranks are summed (all-reduce SUM).
+- the partial FP32 weight gradients of the ranks are summed (all-reduce SUM);
+  on NCCL it is issued as soon as the wgrad GEMM is done and overlaps the
+  dgrad half of the backward pass.
 
 Stochastic rounding draws are keyed by the element's index in the whole
 batch (nvfp4_quantize_rows with row0 = rank * T_local), so every rank's
@@ -31,9 +33,14 @@ class DataParallelLinear:
     The quantized operands live in buffers owned by the object (the same
     operands nvfp4_linear_fwd keeps in its workspace); forward() must run
     before backward() for the same batch.
+
+    timer: optional callable timer(kind, fn) that runs fn() (one library call
+    or one collective) and may record CUDA events around it; kinds name the
+    kernel ("amax_both", "quant_row", "gemm_fprop", ...) or the collective
+    ("allreduce_amax", "allreduce_dw").
     """
 
-    def __init__(self, T_local, Cin, Cout, device, group=None):
+    def __init__(self, T_local, Cin, Cout, device, group=None, timer=None):
         if T_local % 16 or Cin % 16 or Cout % 16:
             raise ValueError("T_local, Cin and Cout must be multiples of 16")
         self.group = group
@@ -41,6 +48,7 @@ class DataParallelLinear:
         self.world = dist.get_world_size(group) if dist.is_initialized() else 1
         self.T, self.Cin, self.Cout = T_local, Cin, Cout
         self.row0 = self.rank * T_local
+        self.timer = timer
         dev = torch.device(device)
         q = api.empty_qtensor
         self.x_row, self.x_col = q(T_local, Cin, dev), q(Cin, T_local, dev)
@@ -49,6 +57,9 @@ class DataParallelLinear:
         self.amax_x = torch.zeros(2, dtype=torch.float32, device=dev)   # [max|X|, max|Q X|]
         self.amax_w = torch.zeros(1, dtype=torch.float32, device=dev)
         self.amax_dy = torch.zeros(2, dtype=torch.float32, device=dev)  # [max|dY|, max|Q dY|]
+
+    def _do(self, kind, fn):
+        return self.timer(kind, fn) if self.timer is not None else fn()
 
     def _all_reduce(self, t, op):
         if self.world == 1:
@@ -64,23 +75,41 @@ class DataParallelLinear:
     def forward(self, X, W, Y=None):
         """Y[T_local, Cout] = X W^T (BF16) for this rank's tokens."""
         assert X.shape == (self.T, self.Cin) and W.shape == (self.Cout, self.Cin)
-        api.amax(X, rht=2, out=self.amax_x)
-        self._all_reduce(self.amax_x, dist.ReduceOp.MAX)
-        api.amax(W, out=self.amax_w)
-        api.quantize(X, api.ROW, self.amax_x[0:1], row_out=self.x_row, row0=self.row0)
-        api.quantize(W, api.TWO_D, self.amax_w, row_out=self.w_row, col_out=self.w_col)
-        api.quantize(X, api.COL, self.amax_x[1:2], rht=True, col_out=self.x_col, row0=self.row0)
-        return api.gemm(self.x_row, self.w_row, api.OUT_BF16, out=Y)
+        d = self._do
+        d("amax_both", lambda: api.amax(X, rht=2, out=self.amax_x))
+        if self.world > 1:
+            d("allreduce_amax", lambda: self._all_reduce(self.amax_x, dist.ReduceOp.MAX))
+        d("quant_row", lambda: api.quantize(X, api.ROW, self.amax_x[0:1], row_out=self.x_row, row0=self.row0))
+        d("amax", lambda: api.amax(W, out=self.amax_w))
+        d("quant_2d", lambda: api.quantize(W, api.TWO_D, self.amax_w, row_out=self.w_row, col_out=self.w_col))
+        Y = d("gemm_fprop", lambda: api.gemm(self.x_row, self.w_row, api.OUT_BF16, out=Y))
+        d("quant_col_rht", lambda: api.quantize(X, api.COL, self.amax_x[1:2], rht=True, col_out=self.x_col,
+                                                row0=self.row0))
+        return Y
 
     def backward(self, dY, seed, dX=None, dW=None):
-        """(dX[T_local, Cin] BF16, dW[Cout, Cin] FP32 summed over the ranks)."""
+        """(dX[T_local, Cin] BF16, dW[Cout, Cin] FP32 summed over the ranks).
+
+        The wgrad half runs first, so that on NCCL the all-reduce of dW runs on
+        the communicator's stream while the dY row copy and the dgrad GEMM
+        compute; the call returns once both are done (stream order)."""
         assert dY.shape == (self.T, self.Cout)
-        api.amax(dY, rht=2, out=self.amax_dy)
-        self._all_reduce(self.amax_dy, dist.ReduceOp.MAX)
-        api.quantize(dY, api.ROW, self.amax_dy[0:1], sr=True, seed=seed, row_out=self.dy_row, row0=self.row0)
-        api.quantize(dY, api.COL, self.amax_dy[1:2], rht=True, sr=True, seed=seed, col_out=self.dy_col,
-                     row0=self.row0)
-        dX = api.gemm(self.dy_row, self.w_col, api.OUT_BF16, out=dX)
-        dW = api.gemm(self.dy_col, self.x_col, api.OUT_F32, out=dW)
-        self._all_reduce(dW, dist.ReduceOp.SUM)
+        d = self._do
+        d("amax_both", lambda: api.amax(dY, rht=2, out=self.amax_dy))
+        if self.world > 1:
+            d("allreduce_amax", lambda: self._all_reduce(self.amax_dy, dist.ReduceOp.MAX))
+        d("quant_col_rht_sr", lambda: api.quantize(dY, api.COL, self.amax_dy[1:2], rht=True, sr=True, seed=seed,
+                                                   col_out=self.dy_col, row0=self.row0))
+        dW = d("gemm_wgrad", lambda: api.gemm(self.dy_col, self.x_col, api.OUT_F32, out=dW))
+        pending = None
+        if self.world > 1:
+            if dist.get_backend(self.group) == "nccl":
+                pending = dist.all_reduce(dW, op=dist.ReduceOp.SUM, group=self.group, async_op=True)
+            else:
+                d("allreduce_dw", lambda: self._all_reduce(dW, dist.ReduceOp.SUM))
+        d("quant_row_sr", lambda: api.quantize(dY, api.ROW, self.amax_dy[0:1], sr=True, seed=seed,
+                                               row_out=self.dy_row, row0=self.row0))
+        dX = d("gemm_dgrad", lambda: api.gemm(self.dy_row, self.w_col, api.OUT_BF16, out=dX))
+        if pending is not None:
+            d("allreduce_dw_wait", pending.wait)   # the current stream waits for the all-reduce
         return dX, dW

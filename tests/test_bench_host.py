@@ -1,10 +1,11 @@
 """Host-side logic of bench.py, CPU only: the clock record that decides whether
 a run is kept (samples outside the timed region ignored, throttle reasons
-collected, median clock), the GEMM traffic figure that is reported only while
-the kernel source still matches the ncu capture, and the config object both
-arms print."""
+collected, median clock), the GEMM profile figures that are reported only while
+the kernel source still matches the ncu capture, the roofline peak, and the
+config object both arms print."""
 import datetime
 import hashlib
+import json
 import os
 import re
 
@@ -56,28 +57,45 @@ def test_clock_summary_without_samples(tmp_path):
     assert c.summary()["reasons"] == ["no samples"]
 
 
-def test_gemm_traffic_is_reported_only_for_the_profiled_source(tmp_path, monkeypatch):
+def test_gemm_profile_is_reported_only_for_the_profiled_source(tmp_path, monkeypatch):
     root = tmp_path
     (root / "profiles").mkdir()
     (root / "nvfp4_bit_microscaled_b200" / "csrc").mkdir(parents=True)
     src = b"// kernel source\n"
     (root / "nvfp4_bit_microscaled_b200" / "csrc" / "gemm.cu").write_bytes(src)
-    prof = root / "profiles" / "gemm_nvf4_full.md"
-    prof.write_text(f"traffic_bytes_per_launch: 1234567\ngemm_source_sha256: {hashlib.sha256(src).hexdigest()}\n")
+    prof = {"traffic_bytes_per_launch": 1234567, "tensor_pipe_pct": 71.5,
+            "gemm_source_sha256": hashlib.sha256(src).hexdigest()}
+    (root / "profiles" / "gemm_traffic.json").write_text(json.dumps(prof))
     monkeypatch.setattr(bench, "ROOT", str(root))
-    assert bench.gemm_traffic_from_profile() == 1234567.0
+    got = bench.gemm_profile()
+    assert got["traffic_bytes_per_launch"] == 1234567 and got["tensor_pipe_pct"] == 71.5
     (root / "nvfp4_bit_microscaled_b200" / "csrc" / "gemm.cu").write_bytes(src + b"// changed\n")
-    assert bench.gemm_traffic_from_profile() is None
+    assert bench.gemm_profile() is None
 
 
-def test_committed_gemm_profile_parses():
-    text = open(os.path.join(bench.ROOT, "profiles", "gemm_nvf4_full.md")).read()
-    assert re.search(r"traffic_bytes_per_launch:\s*[0-9]+", text)
-    assert re.search(r"gemm_source_sha256:\s*[0-9a-f]{64}", text)
+def test_committed_gemm_profile_is_well_formed():
+    path = os.path.join(bench.ROOT, bench.GEMM_PROFILE)
+    if not os.path.exists(path):
+        return
+    prof = json.load(open(path))
+    assert prof["traffic_bytes_per_launch"] > 0 and 0 < prof["tensor_pipe_pct"] <= 100
+    assert re.fullmatch(r"[0-9a-f]{64}", prof["gemm_source_sha256"])
+    assert str(bench.WORKLOAD["T"]) in prof["workload"]
 
 
 def test_both_arms_print_the_same_config():
     c1, c8 = bench.workload_config(1), bench.workload_config(8)
     assert c1["T"] == bench.WORKLOAD["T"] and c1["Cin"] == bench.WORKLOAD["Cin"]
     assert c1["Cout"] == bench.WORKLOAD["Cout"]
-    assert c8["parallelism"].endswith("x8") and c1["workload"] == c8["workload"]
+    assert c8["parallelism"].startswith("dp8") and c1["workload"] == c8["workload"]
+
+
+def test_headline_is_the_largest_configuration():
+    work = {k: w["T"] * w["Cin"] * w["Cout"] for k, w in bench.WORKLOADS.items()}
+    assert bench.HEADLINE == max(work, key=work.get)
+
+
+def test_fp4_roofline_uses_the_burst_bf16_figure():
+    peaks = {"hbm_gbs": 6457.1, "bf16_tflops": 1698.2, "bf16_tflops_sustained": 1430.9}
+    v, src = bench.fp4_peak(peaks, "measured")
+    assert v == 4 * 1698.2 and "burst" in src

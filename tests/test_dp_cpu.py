@@ -91,7 +91,8 @@ def _worker(rank, port, out_dir):
     import oracle as O
     from nvfp4_bit_microscaled_b200 import dp
 
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    if port is not None:                 # mp.spawn; under torchrun the launcher set MASTER_*
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=WORLD)
     dp.api = _OracleApi(O)
     X, W, dY = _inputs()
@@ -111,8 +112,25 @@ def _worker(rank, port, out_dir):
 
 
 def test_data_parallel_linear_equals_whole_batch(tmp_path):
-    import oracle as O
     mp.spawn(_worker, args=(_free_port(), str(tmp_path)), nprocs=WORLD, join=True)
+    _check(tmp_path)
+
+
+def test_data_parallel_linear_under_torchrun(tmp_path):
+    # the launch the multi-GPU bench uses: torchrun, one process per rank, env:// rendezvous
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node", str(WORLD),
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), os.path.abspath(__file__),
+           str(tmp_path)]
+    r = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    _check(tmp_path)
+
+
+def _check(tmp_path):
+    import oracle as O
     X, W, dY = _inputs()
     ax, axr, ag, agr = O.amax(X), O.amax_rht(X), O.amax(dY), O.amax_rht(dY)
     gs = lambda a: float(O.global_scales(a)[1])
@@ -137,3 +155,8 @@ def test_data_parallel_linear_equals_whole_batch(tmp_path):
         assert np.array_equal(r["dy_col_codes"], cgc[:, rows]) and np.array_equal(r["dy_col_sf"], sgc[:, blocks])
         assert np.array_equal(r["Y"], Y[rows]) and np.array_equal(r["dX"], dX[rows])
         assert np.all(np.abs(r["dW"] - dW) <= 1e-12 * absum + 1e-300)           # sum of two partial FP64 GEMMs
+
+
+if __name__ == "__main__":        # one rank under torchrun (test_data_parallel_linear_under_torchrun)
+    import sys
+    _worker(int(os.environ["RANK"]), None, sys.argv[1])
