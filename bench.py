@@ -2,8 +2,8 @@
 
 One step = one full pass of the hot path over one batch, through the
 data-parallel linear layer (nvfp4_bit_microscaled_b200.dp): forward (amax and
-RHT amax of X, X row quantize, W amax, W 2D quantize, fprop GEMM, X column
-quantize with RHT) and backward (amax and RHT amax of dY, dY row quantize with
+RHT amax of X, X row copy and RHT column copy from one read of X, W amax, W 2D
+quantize, fprop GEMM) and backward (amax and RHT amax of dY, dY row quantize with
 SR, dgrad GEMM, dY column quantize with RHT + SR, wgrad GEMM), with the
 all-reduces of the amaxes (MAX) and of dW (SUM) when there is more than one
 rank.  Inputs are seeded synthetic BF16 tensors resident in HBM.
@@ -194,8 +194,8 @@ class EventTimer:
         return out
 
 
-KERNELS_PER_STEP = 11  # 3 amax + 5 quantize + 3 GEMM kernels (no scale padding at these shapes)
-QUANT_KINDS = ("quant_row", "quant_2d", "quant_col_rht", "quant_row_sr", "quant_col_rht_sr")
+KERNELS_PER_STEP = 10  # 3 amax + 4 quantize + 3 GEMM kernels (no scale padding at these shapes)
+QUANT_KINDS = ("quant_rowcol_rht", "quant_2d", "quant_row_sr", "quant_col_rht_sr")
 
 
 def kernel_bytes(T, Ci, Co):
@@ -204,9 +204,8 @@ def kernel_bytes(T, Ci, Co):
     return {
         "amax": 2.0 * Ci * Co,
         "amax_both": 2.0 * (T * Ci + T * Co),
-        "quant_row": 2.0 * T * Ci + q(T, Ci),
+        "quant_rowcol_rht": 2.0 * T * Ci + 2 * q(T, Ci),      # X read once, row copy + RHT column copy
         "quant_2d": 2.0 * Co * Ci + 2 * q(Co, Ci),
-        "quant_col_rht": 2.0 * T * Ci + q(T, Ci),
         "quant_row_sr": 2.0 * T * Co + q(T, Co),
         "quant_col_rht_sr": 2.0 * T * Co + q(T, Co),
     }
@@ -522,7 +521,7 @@ def workload_config(world):
     """The config object both arms print: the headline workload."""
     T, Ci, Co = WORKLOAD["T"], WORKLOAD["Cin"], WORKLOAD["Cout"]
     return {
-        "workload": WORKLOAD["desc"] + "; 3 GEMMs, 3 amax, 5 quantize kernels per step",
+        "workload": WORKLOAD["desc"] + "; 3 GEMMs, 3 amax, 4 quantize kernels per step",
         "T": T, "Cin": Ci, "Cout": Co,
         "parallelism": f"dp{world}" + (" (NCCL all-reduce of amaxes and dW)" if world > 1 else ""),
         "l2": f"inputs larger than L2 (X {2 * T * Ci / 1e6:.0f} MB, W {2 * Co * Ci / 1e6:.0f} MB, "
@@ -564,7 +563,7 @@ def run_reference(args, rank, world):
 
 
 CASES = ("gemm", "gemm_amax", "amax", "amax_rht", "amax_both", "quant_row", "quant_row_sr", "quant_2d", "quant_col_rht",
-         "quant_col_rht_sr", "mx_gemm", "mx_quant_row")
+         "quant_col_rht_sr", "quant_rowcol_rht", "mx_gemm", "mx_quant_row")
 
 
 def _event_ms(fn, reps):
@@ -688,6 +687,12 @@ def run_case(args):
             q = api.empty_qtensor(R, C, dev)
             sr = args.case.endswith("sr")
             fn, work = (lambda: api.quantize(x, api.ROW, amax, sr=sr, seed=1, row_out=q)), 2.0 * R * C + qbytes
+        elif args.case == "quant_rowcol_rht":
+            a2 = torch.zeros(2, dtype=torch.float32, device=dev)
+            api.amax(x, rht=2, out=a2)
+            qr, qc = api.empty_qtensor(R, C, dev), api.empty_qtensor(C, R, dev)
+            fn, work = (lambda: api.quantize(x, api.ROWCOL, a2, rht=True, row_out=qr, col_out=qc)), \
+                2.0 * R * C + 2 * qbytes
         elif args.case == "quant_2d":
             qr, qc = api.empty_qtensor(R, C, dev), api.empty_qtensor(C, R, dev)
             fn, work = (lambda: api.quantize(x, api.TWO_D, amax, row_out=qr, col_out=qc)), 2.0 * R * C + 2 * qbytes

@@ -104,12 +104,17 @@ nvfp4_status nvfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht
  *   x          device BF16 [R, C], pitch ld (ld % 8 == 0).
  *   mode       NVFP4_ROW: row_out gets rows = R, cols = C (C % 16 == 0).
  *              NVFP4_COL: col_out gets rows = C, cols = R (R % 16 == 0, C % 4 == 0).
- *              NVFP4_ROWCOL: both of the above (rht must be 0).
+ *              NVFP4_ROWCOL: both of the above.  Without SR one kernel writes
+ *              both copies from one read of x.  rht = 1 makes the column copy
+ *              the RHT copy: the row copy is then scaled by amax_dev[0] and the
+ *              column copy by amax_dev[1] (the two floats nvfp4_amax(rht = 2)
+ *              writes); with rht = 0 both use amax_dev[0].
  *              NVFP4_2D: 16x16 blocks, R % 16 == 0 and C % 16 == 0; row_out
  *              (rows R, cols C) and/or col_out (rows C, cols R) -- the two
  *              hold the same codes, transposed, with the 16x16 scale repeated
  *              over the 16 rows it covers.
- *   rht        1: apply Q along R before quantizing (COL mode only).
+ *   rht        1: apply Q along R before quantizing the column copy (COL and
+ *              ROWCOL modes only).
  *   sr         1: stochastic rounding (ROW, COL, ROWCOL; not 2D).  The word of
  *              element (r, c) is word ((r*C + c) & 3) of Philox4x32-10 with
  *              key = seed and counter = ((r*C + c) >> 2, domain, 0), domain 0
@@ -120,9 +125,9 @@ nvfp4_status nvfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht
  *   row_out / col_out  caller-filled descriptors (may be NULL when the mode
  *              does not produce that copy); rows/cols must match the above.
  *              Their global_scale receives s_g.
- * Combinations the method excludes return NVFP4_ERR_UNSUPPORTED: RHT on a row
- * copy or in 2D mode (the RHT is for the Wgrad inputs), SR in 2D mode (SR is
- * for gradients; weights round to nearest).
+ * Combinations the method excludes return NVFP4_ERR_UNSUPPORTED: RHT in ROW or
+ * 2D mode (the RHT is for the Wgrad inputs, whose blocks run along the
+ * tokens), SR in 2D mode (SR is for gradients; weights round to nearest).
  */
 nvfp4_status nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, nvfp4_mode mode, int rht, int sr,
                             uint64_t seed, const float* amax_dev, const nvfp4_tensor* row_out,
@@ -207,9 +212,9 @@ nvfp4_status nvfp4_mx_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D
  * Workspace (device, caller-owned, nvfp4_linear_workspace_bytes bytes) holds
  * the quantized operands; linear_fwd leaves in it what linear_bwd needs.
  *
- * nvfp4_linear_fwd: amax(X) -> X row copy (RN); amax(W) -> W 2D (row + column
- *   copies, RN); Y = gemm(Xq, Wq) in BF16; amax_rht(X) -> X column copy with
- *   RHT (RN), kept for wgrad.
+ * nvfp4_linear_fwd: amax and RHT amax of X (one pass) -> X row copy (RN) and X
+ *   column copy with RHT (RN, kept for wgrad) from one read of X; amax(W) ->
+ *   W 2D (row + column copies, RN); Y = gemm(Xq, Wq) in BF16.
  * nvfp4_linear_bwd: amax(dY) -> dY row copy with SR (seed); dX = gemm(dYq, W^T
  *   column copy) in BF16; amax_rht(dY) -> dY column copy with RHT and SR
  *   (seed); dW = gemm(dY^T q, X^T q) in FP32.
@@ -232,10 +237,11 @@ nvfp4_status nvfp4_linear_bwd(const void* dY, int64_t T, int64_t Cin, int64_t Co
  * every device allocation.  Instead of a caller workspace it uses one scratch
  * area of NVFP4_NOALLOC_SCRATCH_BYTES inside the library image (a __device__
  * array that every GPU which loads the library holds until process exit).
- *   - Computes Y exactly as nvfp4_linear_fwd does (the same kernels in the
- *     same order), bit for bit.  It skips the one step whose result only
- *     nvfp4_linear_bwd reads (the X column copy for wgrad): there is no
- *     allocation-free backward to read it.  X, W, Y as in nvfp4_linear_fwd.
+ *   - Computes Y bit for bit as nvfp4_linear_fwd does.  It skips the X
+ *     column copy for wgrad, which only nvfp4_linear_bwd reads (there is no
+ *     allocation-free backward), and so makes X's row copy with the row
+ *     quantizer alone: the same codes and scales.  X, W, Y as in
+ *     nvfp4_linear_fwd.
  *   - T, Cin, Cout: multiples of 64, each below 2^31 (NVFP4_ERR_SHAPE).
  *   - Returns NVFP4_ERR_WORKSPACE, before enqueuing anything, when the part
  *     of the linear workspace the forward uses (the scalars, the X row copy

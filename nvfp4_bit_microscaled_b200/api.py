@@ -68,11 +68,15 @@ def quantize(x, mode, amax_dev, rht=False, sr=False, seed=0, row_out=None, col_o
     """BF16 [R, C] -> (row copy, column copy); a copy the mode does not make is None.
 
     In TWO_D mode both copies are made unless row_out or col_out is False.
+    ROWCOL with rht: the row copy is scaled by amax_dev[0] and the RHT column
+    copy by amax_dev[1] (the two floats amax(x, rht=2) returns).
     row0 != 0 (nvfp4_quantize_rows): x is rows row0 .. of a larger tensor, and
     the SR draws are those of the whole tensor's elements.
     """
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     R, C = x.shape
+    if mode == ROWCOL and rht:
+        assert amax_dev.numel() >= 2, "ROWCOL with rht takes [amax of x, amax of Q x]"
     want_row = mode in (ROW, ROWCOL) or (mode == TWO_D and row_out is not False)
     want_col = mode in (COL, ROWCOL) or (mode == TWO_D and col_out is not False)
     if want_row and not isinstance(row_out, QTensor):

@@ -9,6 +9,8 @@
 // Both kernels are HBM-bound: 2 bytes read per element, one 4-byte result.
 // The result is combined across CTAs with an integer atomicMax on the float's
 // bit pattern (non-negative floats order like their bit patterns).
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -126,6 +128,26 @@ __global__ void __launch_bounds__(256, 3) amax_rht_kernel(const uint16_t* __rest
   }
 }
 
+// CTAs of `kernel` (256 threads) that are resident on one SM at once, per
+// device, queried once: the grid-stride amax kernels launch exactly one wave.
+template <class Kernel>
+int resident_ctas(Kernel kernel, int* cache) {
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, 256, 0) != cudaSuccess || n < 1) {
+      (void)cudaGetLastError();
+      n = 1;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+int g_occ_rht_both[64], g_occ_rht[64], g_occ_flat[64];
+
 cudaError_t launch_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht, float* amax_dev, int num_sms,
                         cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(amax_dev, 0, (rht == 2 ? 2 : 1) * sizeof(float), s);
@@ -135,7 +157,10 @@ cudaError_t launch_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht
   if (rht) {
     const int64_t items = (R / 16) * (C / 4);
     const int64_t blocks = (items + 255) / 256;
-    const int grid = static_cast<int>(blocks < 6LL * num_sms ? blocks : 6LL * num_sms);
+    const int64_t wave = static_cast<int64_t>(num_sms) *
+                         (rht == 2 ? resident_ctas(amax_rht_kernel<true>, g_occ_rht_both)
+                                   : resident_ctas(amax_rht_kernel<false>, g_occ_rht));
+    const int grid = static_cast<int>(blocks < wave ? blocks : wave);
     if (rht == 2)
       amax_rht_kernel<true><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), R, C, ld, out);
     else
@@ -143,7 +168,8 @@ cudaError_t launch_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht
   } else if (ld == C && (R * C) % 8 == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
     const int64_t n8 = R * C / 8;
     const int64_t blocks = (n8 + 255) / 256;
-    const int grid = static_cast<int>(blocks < 4LL * num_sms ? blocks : 4LL * num_sms);
+    const int64_t wave = static_cast<int64_t>(num_sms) * resident_ctas(amax_flat_kernel, g_occ_flat);
+    const int grid = static_cast<int>(blocks < wave ? blocks : wave);
     amax_flat_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), n8, out);
   } else {
     const int64_t blocks = (R + 7) / 8;

@@ -134,16 +134,20 @@ nvfp4_status linear_forward(const void* X, const void* W, int64_t T, int64_t Cin
   // fprop operands: X row-wise (RN), W 2D (RN) with its transposed copy for dgrad
   // one pass over X gives both its amax (row copy) and its RHT amax (column copy)
   if ((st = nvfp4_amax(X, T, Cin, Cin, 2, amax + kAmaxX, stream)) != NVFP4_OK) return st;
-  if ((st = nvfp4_quantize(X, T, Cin, Cin, NVFP4_ROW, 0, 0, 0, amax + kAmaxX, &xr, nullptr, stream)) != NVFP4_OK)
+  if (keep_wgrad) {
+    // the X row copy (fprop) and the X^T copy with the RHT along tokens, saved
+    // for wgrad, from one read of X; amax + kAmaxX holds [max|X|, max|Q X|]
+    const nvfp4_tensor xc = ws_tensor(ws, L, 3);
+    if ((st = nvfp4_quantize(X, T, Cin, Cin, NVFP4_ROWCOL, 1, 0, 0, amax + kAmaxX, &xr, &xc, stream)) != NVFP4_OK)
+      return st;
+  } else if ((st = nvfp4_quantize(X, T, Cin, Cin, NVFP4_ROW, 0, 0, 0, amax + kAmaxX, &xr, nullptr, stream)) !=
+             NVFP4_OK) {
     return st;
+  }
   if ((st = nvfp4_amax(W, Cout, Cin, Cin, 0, amax + kAmaxW, stream)) != NVFP4_OK) return st;
   if ((st = nvfp4_quantize(W, Cout, Cin, Cin, NVFP4_2D, 0, 0, 0, amax + kAmaxW, &wr, &wc, stream)) != NVFP4_OK)
     return st;
-  if ((st = nvfp4_gemm(&xr, &wr, Y, NVFP4_OUT_BF16, Cout, stream)) != NVFP4_OK) return st;
-  if (!keep_wgrad) return NVFP4_OK;
-  // wgrad operand saved for the backward pass: X^T with the RHT along tokens (RN)
-  const nvfp4_tensor xc = ws_tensor(ws, L, 3);
-  return nvfp4_quantize(X, T, Cin, Cin, NVFP4_COL, 1, 0, 0, amax + kAmaxXr, nullptr, &xc, stream);
+  return nvfp4_gemm(&xr, &wr, Y, NVFP4_OUT_BF16, Cout, stream);
 }
 
 }  // namespace nvfp4
@@ -253,7 +257,7 @@ static nvfp4_status quantize_checked(const void* x, int64_t R, int64_t C, int64_
     return NVFP4_ERR_INVALID_ARG;
   if (R <= 0 || C <= 0 || ld < C) return NVFP4_ERR_SHAPE;
   if (!aligned16(x) || ld % 8) return NVFP4_ERR_ALIGN;
-  if (rht && mode != NVFP4_COL) return NVFP4_ERR_UNSUPPORTED;
+  if (rht && mode != NVFP4_COL && mode != NVFP4_ROWCOL) return NVFP4_ERR_UNSUPPORTED;
   if (sr && mode == NVFP4_2D) return NVFP4_ERR_UNSUPPORTED;
   if (row0 < 0 || row0 % 16 || row0 >= (int64_t(1) << 40)) return NVFP4_ERR_SHAPE;
   if (row0 && row0 + R > (int64_t(1) << 62) / C) return NVFP4_ERR_SHAPE;  // (row0 + R) * C stays in int64
@@ -278,13 +282,21 @@ static nvfp4_status quantize_checked(const void* x, int64_t R, int64_t C, int64_
                                want_col ? col_out->global_scale : nullptr, di.sms, s);
     return cuda_status(e);
   }
+  // ROWCOL with RHT: the row copy takes amax_dev[0], the RHT column copy amax_dev[1]
+  const float* amax_col = (mode == NVFP4_ROWCOL && rht) ? amax_dev + 1 : amax_dev;
+  if (mode == NVFP4_ROWCOL && !sr) {   // both copies from one read of x
+    e = nvfp4::launch_quant_rowcol(x, R, C, ld, amax_dev, amax_col, rht, row_out->data, row_out->scales,
+                                   row_out->global_scale, col_out->data, col_out->scales, col_out->global_scale,
+                                   di.sms, s);
+    return cuda_status(e);
+  }
   if (want_row) {
     e = nvfp4::launch_quant_row(x, R, C, ld, amax_dev, sr, seed, row0 * C, row_out->data, row_out->scales,
                                 row_out->global_scale, di.sms, s);
     if (e != cudaSuccess) return cuda_status(e);
   }
   if (want_col) {
-    e = nvfp4::launch_quant_col(x, R, C, ld, amax_dev, rht, sr, seed, row0 * C, col_out->data,
+    e = nvfp4::launch_quant_col(x, R, C, ld, amax_col, rht, sr, seed, row0 * C, col_out->data,
                                 col_out->scales, col_out->global_scale, di.sms, s);
     if (e != cudaSuccess) return cuda_status(e);
   }

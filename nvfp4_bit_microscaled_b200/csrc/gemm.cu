@@ -369,6 +369,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 // tensor-pipe time.
 // ===========================================================================
 constexpr int P_STAGES = 5;
+constexpr int P_NUM_THREADS = NUM_THREADS;
 constexpr uint32_t P_A_BYTES = 128 * BK_BYTES;                 // 16 KiB (own A rows)
 constexpr uint32_t P_B_BYTES = 128 * BK_BYTES;                 // 16 KiB (own half of B)
 constexpr uint32_t P_SFA_BYTES = KB_PER_STAGE * 512;           // 2 KiB
@@ -422,7 +423,7 @@ __device__ __forceinline__ void pair_mma_step(uint32_t acc, uint64_t adesc, uint
 // names its byte pair of the scale cell (see mma_mxf4_pair).  AMAX: the
 // epilogue also reduces max |D| into *amax_out (see epilogue_amax_commit).
 template <bool MX, bool AMAX>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(P_NUM_THREADS, 1)
 gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmD, const uint8_t* __restrict__ sfa,
                       const uint8_t* __restrict__ sfb, const float* __restrict__ gsa,
@@ -565,7 +566,7 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     }
     tc_commit_pair(mma_done);
     mbar_wait(mma_done, 0, kErrWaitAccFull);
-  } else if (warp >= SF_WARP0) {
+  } else if (warp >= SF_WARP0 && warp < SF_WARP0 + NUM_SF_WARPS) {
     // ------------------------------------------------------------ scale warps (both CTAs)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int stage = 0;
@@ -611,7 +612,7 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       }
       if (!ok) { *abort_flag = 1; break; }
     }
-  } else if (warp >= EPI_WARP0) {
+  } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + NUM_EPI_WARPS) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     // Warp w reads TMEM lanes 32*(w%4) .. +31 (its rows) and 128 accumulator
     // columns, scales by alpha, and stores 32-row x 128-byte boxes (64 BF16 or
@@ -636,71 +637,82 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       const int row0 = tm * 256 + 128 * static_cast<int>(rank) + quarter * 32;
       const int col_base = tn * 256 + col_half * 128;
       float tile_max = 0.0f;
-      if (out_bf16) {
+      const uint32_t acc = tmem + lane_base + ACC_COL + col_half * 128;
+      // alpha * accumulator -> BF16 pairs in place: word e of r becomes the pair
+      // (2e, 2e + 1) (e <= 2e, so nothing is overwritten before it is read);
+      // also the running |D| maximum
+      auto to_bf16 = [&](uint32_t (&r)[32]) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {  // two boxes of 64 columns
-          uint32_t packed[32];
-#pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(tmem + lane_base + ACC_COL + col_half * 128 + h * 64 + ch * 32, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float v0 = __fmul_rn(__uint_as_float(r[2 * e]), alpha);
-              const float v1 = __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha);
-              if (AMAX) tile_max = fmaxf(tile_max, fmaxf(fabsf(v0), fabsf(v1)));
-              __nv_bfloat162 v = __floats2bfloat162_rn(v0, v1);
-              packed[16 * ch + e] = *reinterpret_cast<uint32_t*>(&v);
-            }
-          }
-          if (h == 1) {  // every accumulator column of this warp is in registers
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty_l);
-          }
-          if (lane == 0) bulk_wait_read_all();  // the previous box has left the staging buffer
-          __syncwarp();
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(my_row + 16 * (j ^ sw)) =
-                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && row0 < M && col_base + 64 * h < N) {  // boxes past the matrix: nothing to store
-            tma_store_2d(&tmD, stg, col_base + 64 * h, row0);
-            bulk_commit_group();
-          }
+        for (int e = 0; e < 16; ++e) {
+          const float v0 = __fmul_rn(__uint_as_float(r[2 * e]), alpha);
+          const float v1 = __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha);
+          if (AMAX) tile_max = fmaxf(tile_max, fmaxf(fabsf(v0), fabsf(v1)));
+          __nv_bfloat162 v = __floats2bfloat162_rn(v0, v1);
+          r[e] = *reinterpret_cast<uint32_t*>(&v);
         }
+      };
+      // one 32-row x 128-byte box (16 words from lo, then 16 from hi) through the staging buffer
+      auto store_box = [&](const uint32_t* lo, const uint32_t* hi, int col) {
+        if (lane == 0) bulk_wait_read_all();  // the previous box has left the staging buffer
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t* w = j < 4 ? lo + 4 * j : hi + 4 * (j - 4);
+          *reinterpret_cast<uint4*>(my_row + 16 * (j ^ sw)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < M && col < N) {  // boxes past the matrix: nothing to store
+          tma_store_2d(&tmD, stg, col, row0);
+          bulk_commit_group();
+        }
+      };
+      auto hand_back = [&]() {  // every accumulator column of this warp is in registers
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty_l);
+      };
+      if (out_bf16) {
+        // Two boxes of 64 columns, each read with two loads and one wait; the
+        // accumulator goes back as soon as the second box is in registers.
+        uint32_t ra[32], rb[32];
+        tmem_ld_32x32b_x32(acc + 0, ra);
+        tmem_ld_32x32b_x32(acc + 32, rb);
+        tmem_ld_wait();
+        to_bf16(ra);
+        to_bf16(rb);
+        store_box(ra, rb, col_base);
+        tmem_ld_32x32b_x32(acc + 64, ra);
+        tmem_ld_32x32b_x32(acc + 96, rb);
+        tmem_ld_wait();
+        hand_back();
+        to_bf16(ra);
+        to_bf16(rb);
+        store_box(ra, rb, col_base + 64);
       } else {
-#pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {  // four boxes of 32 columns
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + ACC_COL + col_half * 128 + ch * 32, r);
-          tmem_ld_wait();
-          if (ch == 3) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty_l);
-          }
+        // Four boxes of 32 columns, read two at a time (two loads, one wait);
+        // the accumulator goes back once the last two are in registers.
+        uint32_t ra[32], rb[32];
+        auto fp32_box = [&](uint32_t (&r)[32], int ch) {
           if (AMAX) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) tile_max = fmaxf(tile_max, fabsf(__fmul_rn(__uint_as_float(r[e]), alpha)));
           }
-          if (lane == 0) bulk_wait_read_all();
-          __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<float4*>(my_row + 16 * (j ^ sw)) = make_float4(
-                __fmul_rn(__uint_as_float(r[4 * j + 0]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 1]), alpha),
-                __fmul_rn(__uint_as_float(r[4 * j + 2]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 3]), alpha));
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && row0 < M && col_base + 32 * ch < N) {
-            tma_store_2d(&tmD, stg, col_base + 32 * ch, row0);
-            bulk_commit_group();
-          }
-        }
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__fmul_rn(__uint_as_float(r[e]), alpha));
+          store_box(r, r + 16, col_base + 32 * ch);
+        };
+        tmem_ld_32x32b_x32(acc + 0, ra);
+        tmem_ld_32x32b_x32(acc + 32, rb);
+        tmem_ld_wait();
+        fp32_box(ra, 0);
+        fp32_box(rb, 1);
+        tmem_ld_32x32b_x32(acc + 64, ra);
+        tmem_ld_32x32b_x32(acc + 96, rb);
+        tmem_ld_wait();
+        hand_back();
+        fp32_box(ra, 2);
+        fp32_box(rb, 3);
       }
       if (AMAX && row0 + lane < M) run_max = fmaxf(run_max, tile_max);
       acc_phase ^= 1u;
@@ -816,7 +828,7 @@ cudaError_t setup_kernel(KernelSetup* cache, Kernel kern, uint32_t smem_bytes, b
     if (cluster_pairs) {
       cudaLaunchConfig_t q = {};
       q.gridDim = dim3(2 * (num_sms / 2));
-      q.blockDim = dim3(NUM_THREADS);
+      q.blockDim = dim3(P_NUM_THREADS);
       q.dynamicSmemBytes = smem_bytes;
       cudaLaunchAttribute qa[1];
       qa[0].id = cudaLaunchAttributeClusterDimension;
@@ -880,7 +892,7 @@ cudaError_t launch_gemm(const void* a_data, const void* a_scales, const float* a
     group_m = group_m < 1 ? 1 : (group_m > num_m ? num_m : group_m);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
-    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.blockDim = dim3(P_NUM_THREADS);
     cfg.dynamicSmemBytes = P_SMEM_BYTES;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

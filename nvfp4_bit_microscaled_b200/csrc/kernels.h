@@ -22,6 +22,13 @@ cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, co
                              int sr, uint64_t seed, int64_t idx0, void* data, void* scales, float* gs_out,
                              int num_sms, cudaStream_t s);
 
+// Row copy (data [R, C/2]) and column copy (data [C, R/2], RHT along R when
+// rht != 0) from one read of x, round to nearest; the row copy is scaled by
+// *amax_row, the column copy by *amax_col.
+cudaError_t launch_quant_rowcol(const void* x, int64_t R, int64_t C, int64_t ld, const float* amax_row,
+                                const float* amax_col, int rht, void* row_data, void* row_scales, float* row_gs,
+                                void* col_data, void* col_scales, float* col_gs, int num_sms, cudaStream_t s);
+
 // MXFP4 row-wise 1x32 quantization: data [R, C/2], UE8M0 scales in the 128x4
 // tile layout with sp = pad4(C/32); writes 1.0 to *gs_out when given.
 cudaError_t launch_mx_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, void* data, void* scales,

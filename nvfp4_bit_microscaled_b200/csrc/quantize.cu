@@ -347,6 +347,121 @@ __global__ void __launch_bounds__(256, 2) quant_col_rn_kernel(const uint16_t* __
 }
 
 // ---------------------------------------------------------------------------
+// Row copy and column copy from one read of x (NVFP4_ROWCOL without SR): the
+// X of a linear layer needs its row copy for fprop and its RHT column copy for
+// wgrad, and two kernels would read it twice.  Warp item: 64 tokens x 128
+// channels, in four bands of 16 rows.  For each band, lane l loads its 4
+// channels of the 16 rows (8-byte loads, 256 coalesced bytes per row per warp)
+// and quantizes their column blocks from registers, as the column kernel does
+// (RHT optional, scaled by the column copy's amax); it also stages the band in
+// shared memory, from which lanes read the band's 16 x 8 row blocks of 16
+// channels (two 16-byte reads each) and quantize them as the row kernel does
+// (scaled by the row copy's amax).  A non-finite amax flags its copy (R25).
+// ---------------------------------------------------------------------------
+constexpr int kBandPitch = 272;   // 256 bytes of a staged row + 16: rows start on different banks
+template <bool RHT>
+__global__ void __launch_bounds__(256, 2) quant_rowcol_kernel(
+    const uint16_t* __restrict__ x, int64_t R, int64_t C, int64_t ld, const float* __restrict__ amax_row_dev,
+    const float* __restrict__ amax_col_dev, uint8_t* __restrict__ row_data, uint8_t* __restrict__ row_sf,
+    int64_t row_sp, float* __restrict__ row_gs, uint8_t* __restrict__ col_data, uint8_t* __restrict__ col_sf,
+    int64_t col_sp, float* __restrict__ col_gs) {
+  __shared__ float r_row[kRTableSize], r_col[kRTableSize];
+  __shared__ __align__(16) uint8_t band[8][16][kBandPitch];
+  const float a_row = __ldg(amax_row_dev), a_col = __ldg(amax_col_dev);
+  const float se_row = encode_scale(a_row), se_col = encode_scale(a_col);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *row_gs = decode_scale(a_row);
+    *col_gs = decode_scale(a_col);
+  }
+  const bool flag_row = !isfinite(a_row), flag_col = !isfinite(a_col);
+  if (flag_row) flag_copy(row_data, R, C >> 1, row_sf, C >> 4, row_sp);
+  if (flag_col) flag_copy(col_data, C, R >> 1, col_sf, R >> 4, col_sp);
+  if (flag_row && flag_col) return;
+  fill_r_table(r_row, se_row);
+  fill_r_table(r_col, se_col);
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  uint8_t (*bw)[kBandPitch] = band[wib];
+  const int64_t S = R >> 4, nq = (S + 3) >> 2, ng = (C + 127) >> 7, items = nq * ng;
+  const int64_t half_r = R >> 1, half_c = C >> 1;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + wib; it < items; it += nwarps) {
+    const int64_t q = it / ng, cw = (it - q * ng) * 128, t0 = q * 64, c0 = cw + 4 * lane;
+    const bool lane_ok = c0 < C;
+    const int nb = static_cast<int>((S - 4 * q) < 4 ? (S - 4 * q) : 4);
+    uint32_t sfw[4] = {0u, 0u, 0u, 0u};
+    for (int tb = 0; tb < nb; ++tb) {
+      const int64_t tbase = t0 + 16 * tb;
+      uint2 raw[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        raw[i] = lane_ok ? __ldcs(reinterpret_cast<const uint2*>(x + (tbase + i) * ld + c0)) : make_uint2(0u, 0u);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) *reinterpret_cast<uint2*>(&bw[i][8 * lane]) = raw[i];
+      if (!flag_col && lane_ok) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {   // column blocks: channel c0 + c, tokens tbase .. + 15
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint32_t w = (c < 2) ? raw[i].x : raw[i].y;
+            v[i] = __uint_as_float((c & 1) ? (w & 0xFFFF0000u) : (w << 16));
+            if (RHT && rht_negates(i)) v[i] = -v[i];  // s_i x_i
+          }
+          float m = 0.0f;
+          if (RHT) {
+            m = __fmul_rn(fwht16_absmax<true>(v), 0.25f);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.25f);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+          }
+          const BlockScale bs = block_scale_t(m, se_col, r_col);
+          sfw[c] |= bs.sf << (8 * tb);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], bs.r);
+          reinterpret_cast<uint2*>(col_data + (c0 + c) * half_r + t0 / 2)[tb] = make_uint2(pack8(v), pack8(v + 8));
+        }
+      }
+      __syncwarp();
+      if (!flag_row) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {   // row blocks: row (lane / 8) + 4j, 16 channels cw + 16 (lane % 8) ..
+          const int i = (lane >> 3) + 4 * j, b = lane & 7;
+          const int64_t cb = cw + 16 * b;
+          const bool ok = cb < C;
+          uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+          if (ok) {
+            v0 = *reinterpret_cast<const uint4*>(&bw[i][32 * b]);
+            v1 = *reinterpret_cast<const uint4*>(&bw[i][32 * b + 16]);
+          }
+          const uint32_t mb = max(absmax_bits8(v0), absmax_bits8(v1));
+          const BlockScale bs = block_scale_t(bf16_bits_to_f32(mb), se_row, r_row);
+          float y[16];
+          unpack8(v0, y);
+          unpack8(v1, y + 8);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) y[e] = __fmul_rn(y[e], bs.r);
+          const uint32_t w0 = pack8(y), w1 = pack8(y + 8);
+          if (ok) *reinterpret_cast<uint2*>(row_data + (tbase + i) * half_c + cb / 2) = make_uint2(w0, w1);
+          // lanes 4k .. 4k+3 hold four consecutive blocks of the row: one scale word
+          uint32_t word = ok ? (bs.sf << (8 * (b & 3))) : 0u;
+          word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+          word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+          if ((lane & 3) == 0 && ok) *reinterpret_cast<uint32_t*>(row_sf + sf_offset(tbase + i, cb >> 4, row_sp)) = word;
+        }
+      }
+      __syncwarp();   // the band buffer is rewritten by the next band
+    }
+    if (!flag_col && lane_ok) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) *reinterpret_cast<uint32_t*>(col_sf + sf_offset(c0 + c, 4 * q, col_sp)) = sfw[c];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // 2D 16x16 (weights).  CTA slab: 64 rows (4 tile rows) x 128 columns (8 tile
 // columns) of W.  Warp w takes tile row w/2 and tile columns 4*(w%2) .. +3;
 // eight lanes share a tile, lane l holding columns 2*(l%8), +1 of tile l/8
@@ -627,6 +742,30 @@ cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, co
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_sf_pad_zero(scales, C, S, s);
+}
+
+cudaError_t launch_quant_rowcol(const void* x, int64_t R, int64_t C, int64_t ld, const float* amax_row,
+                                const float* amax_col, int rht, void* row_data, void* row_scales, float* row_gs,
+                                void* col_data, void* col_scales, float* col_gs, int num_sms, cudaStream_t s) {
+  const int64_t S = R / 16;
+  const int64_t warp_items = ((S + 3) / 4) * ((C + 127) / 128);
+  const int grid = grid_for(warp_items, 8, num_sms, 8);
+  auto* xs = static_cast<const uint16_t*>(x);
+  auto* rd = static_cast<uint8_t*>(row_data);
+  auto* rf = static_cast<uint8_t*>(row_scales);
+  auto* cd = static_cast<uint8_t*>(col_data);
+  auto* cf = static_cast<uint8_t*>(col_scales);
+  const int64_t row_sp = (C / 16 + 3) / 4 * 4, col_sp = (S + 3) / 4 * 4;
+  if (rht)
+    quant_rowcol_kernel<true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_row, amax_col, rd, rf, row_sp, row_gs, cd, cf,
+                                                   col_sp, col_gs);
+  else
+    quant_rowcol_kernel<false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_row, amax_col, rd, rf, row_sp, row_gs, cd, cf,
+                                                    col_sp, col_gs);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if ((e = launch_sf_pad_zero(row_scales, R, C / 16, s)) != cudaSuccess) return e;
+  return launch_sf_pad_zero(col_scales, C, S, s);
 }
 
 cudaError_t launch_mx_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, void* data, void* scales,

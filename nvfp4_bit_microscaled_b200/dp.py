@@ -79,13 +79,12 @@ class DataParallelLinear:
         d("amax_both", lambda: api.amax(X, rht=2, out=self.amax_x))
         if self.world > 1:
             d("allreduce_amax", lambda: self._all_reduce(self.amax_x, dist.ReduceOp.MAX))
-        d("quant_row", lambda: api.quantize(X, api.ROW, self.amax_x[0:1], row_out=self.x_row, row0=self.row0))
+        # X's row copy (fprop) and RHT column copy (wgrad) from one read of X
+        d("quant_rowcol_rht", lambda: api.quantize(X, api.ROWCOL, self.amax_x, rht=True, row_out=self.x_row,
+                                                   col_out=self.x_col, row0=self.row0))
         d("amax", lambda: api.amax(W, out=self.amax_w))
         d("quant_2d", lambda: api.quantize(W, api.TWO_D, self.amax_w, row_out=self.w_row, col_out=self.w_col))
-        Y = d("gemm_fprop", lambda: api.gemm(self.x_row, self.w_row, api.OUT_BF16, out=Y))
-        d("quant_col_rht", lambda: api.quantize(X, api.COL, self.amax_x[1:2], rht=True, col_out=self.x_col,
-                                                row0=self.row0))
-        return Y
+        return d("gemm_fprop", lambda: api.gemm(self.x_row, self.w_row, api.OUT_BF16, out=Y))
 
     def backward(self, dY, seed, dX=None, dW=None):
         """(dX[T_local, Cin] BF16, dW[Cout, Cin] FP32 summed over the ranks).

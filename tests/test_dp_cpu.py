@@ -71,13 +71,16 @@ class _OracleApi:
             row_out.gs = col_out.gs = gs
             return row_out, col_out
         xp = self._padded(x, row0)
-        if mode == self.ROW:
+        if mode in (self.ROW, self.ROWCOL):
             c, s = O.quantize_row(xp, a, sr=sr, seed=seed)
             row_out.codes, row_out.sf, row_out.gs = c[row0:], s[row0:], gs
-        else:
-            c, s = O.quantize_col(xp, a, rht=rht, sr=sr, seed=seed)
-            col_out.codes, col_out.sf, col_out.gs = c[:, row0:], s[:, row0 // 16:], gs
-        assert (row_out or col_out).codes.shape[0 if mode == self.ROW else 1] == R
+            assert row_out.codes.shape[0] == R
+        if mode in (self.COL, self.ROWCOL):
+            # ROWCOL with RHT: the column copy is scaled by the second amax (the RHT one)
+            ac = float(amax_dev[1]) if (mode == self.ROWCOL and rht) else a
+            c, s = O.quantize_col(xp, ac, rht=rht, sr=sr, seed=seed)
+            col_out.codes, col_out.sf, col_out.gs = c[:, row0:], s[:, row0 // 16:], float(O.global_scales(ac)[1])
+            assert col_out.codes.shape[1] == R
         return row_out, col_out
 
     def gemm(self, A, B, out_dtype=0, out=None):

@@ -62,11 +62,14 @@ def test_quantizers_flag_copies_of_nonfinite_tensor(kind):
     assert_q_equal(row_sr, *O.quantize_row(x, a, sr=True, seed=9), a, "row sr")
     _, col = api.quantize(xd, api.COL, ar_dev, rht=True, sr=True, seed=9)
     assert_q_equal(col, *O.quantize_col(x, ar, rht=True, sr=True, seed=9), ar, "col rht sr")
+    rr, rc = api.quantize(xd, api.ROWCOL, api.amax(xd, rht=2), rht=True)
+    assert_q_equal(rr, *O.quantize_row(x, a), a, "rowcol row")
+    assert_q_equal(rc, *O.quantize_col(x, ar, rht=True), ar, "rowcol col")
     r2, c2 = api.quantize(xd, api.TWO_D, a_dev)
     (cr, sr_), (cc, sc) = O.expand_2d(*O.quantize_2d(x, a))
     assert_q_equal(r2, cr, sr_, a, "2d row")
     assert_q_equal(c2, cc, sc, a, "2d col")
-    for q in (row, row_sr, col, r2, c2):
+    for q in (row, row_sr, col, rr, rc, r2, c2):
         assert api.copy_is_flagged(q)
         assert int((q.scales == 0x7F).sum()) == q.rows * (q.cols // 16)   # padding stays 0
 

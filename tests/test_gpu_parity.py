@@ -145,6 +145,31 @@ def test_quantize_rowcol():
     assert_q_equal(col, *O.quantize_col(x, a, sr=True, seed=5), a, "rowcol col")
 
 
+@pytest.mark.parametrize("name,x", _inputs())
+@pytest.mark.parametrize("rht", [False, True])
+def test_quantize_rowcol_one_read(name, x, rht):
+    # ROWCOL without SR: one kernel writes both copies from one read of x; with
+    # RHT the column copy is the RHT copy, scaled by the RHT amax (amax_dev[1])
+    R = x.shape[0] // 16 * 16
+    x = x[:R].contiguous()
+    a, ar = O.amax(x), O.amax_rht(x)
+    amax_dev = api.amax(dev(x), rht=2) if rht else api.amax(dev(x))
+    row, col = api.quantize(dev(x), api.ROWCOL, amax_dev, rht=rht)
+    assert_q_equal(row, *O.quantize_row(x, a), a, f"{name} rowcol row")
+    ac = ar if rht else a
+    assert_q_equal(col, *O.quantize_col(x, ac, rht=rht), ac, f"{name} rowcol col rht={rht}")
+
+
+@pytest.mark.parametrize("R,C", [(64, 128), (80, 144), (16, 4096 + 16), (1040, 272)])
+def test_quantize_rowcol_one_read_tails(R, C):
+    # token counts that are not multiples of 64 and channel counts that are not multiples of 128
+    x = synth.activations(R, C, 44)
+    a, ar = O.amax(x), O.amax_rht(x)
+    row, col = api.quantize(dev(x), api.ROWCOL, api.amax(dev(x), rht=2), rht=True)
+    assert_q_equal(row, *O.quantize_row(x, a), a, f"rowcol row {R}x{C}")
+    assert_q_equal(col, *O.quantize_col(x, ar, rht=True), ar, f"rowcol col {R}x{C}")
+
+
 # ------------------------------------------------------------------ 2D
 @pytest.mark.parametrize("shape", [(128, 256), (48, 80), (208, 336), (16, 16)])
 def test_quantize_2d(shape):
