@@ -89,18 +89,26 @@ def gemm_profile():
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """SM clocks and throttle reasons sampled during the timed region: NVML from a
+    thread every few milliseconds (the timed region can be a fraction of a
+    second), else nvidia-smi at its 200 ms floor.  Reads only; sets nothing."""
 
-    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown", 0x8),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap", 0x4))
+    SMI_FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index, enabled=True):
-        self.gpu_index = gpu_index
+    def __init__(self, device, enabled=True, period_s=0.005):
+        self.device = device              # torch CUDA device index
         self.enabled = enabled
-        self.proc = None
-        self.path = os.path.join(tempfile.gettempdir(), f"nvfp4_bench_clocks_{os.getpid()}_{gpu_index}.csv")
+        self.period = period_s
+        self.samples = []                 # (time, sm MHz, max sm MHz, set of reason names)
+        self.source = None
         self.t0 = self.t1 = None
+        self.proc = self.thread = None
 
     def mark_start(self):
         self.t0 = time.time()
@@ -108,35 +116,45 @@ class ClockSampler:
     def mark_end(self):
         self.t1 = time.time()
 
-    def __enter__(self):
-        if not self.enabled:
-            return self
-        try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
-                 "-i", str(self.gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
-            time.sleep(1.0)          # let the sampler start before the timed region
-        except (OSError, FileNotFoundError):
-            self.proc = None
-        return self
+    # -- NVML
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(self.device)
+        if all(hasattr(p, k) for k in ("pci_domain_id", "pci_bus_id", "pci_device_id")):
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        idx = int(vis.split(",")[self.device]) if vis else self.device
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(idx)
 
-    def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+    def _nvml_loop(self, nv, h, stop):
+        reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        bits = [(n, getattr(nv, attr, v)) for n, attr, v in self.REASONS]
+        clk_max = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not stop.wait(self.period):
             try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.f.close()
+                clk = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                r = reasons_fn(h)
+            except Exception:
+                continue
+            self.samples.append((time.time(), float(clk), float(clk_max), {n for n, b in bits if r & b}))
 
-    def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+    # -- nvidia-smi
+    def _smi_start(self):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        idx = vis.split(",")[self.device] if vis else str(self.device)
+        self.path = os.path.join(tempfile.gettempdir(), f"nvfp4_bench_clocks_{os.getpid()}_{self.device}.csv")
+        self.f = open(self.path, "w")
+        self.proc = subprocess.Popen(
+            ["nvidia-smi", f"--query-gpu={self.SMI_FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+             "-i", idx], stdout=self.f, stderr=subprocess.DEVNULL)
+        time.sleep(1.0)          # let the sampler start before the timed region
+
+    def _smi_read(self):
         import datetime
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        names = [n for n, _, _ in self.REASONS]
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
@@ -147,21 +165,56 @@ class ClockSampler:
                     clk, clk_max = float(parts[2]), float(parts[3])
                 except ValueError:
                     continue
-                if self.t0 is not None and not (self.t0 <= ts <= (self.t1 or ts)):
-                    continue
-                sm.append(clk)
-                smax.append(clk_max)
-                for n, v in zip(names, parts[6:10]):
-                    if v.lower() == "active":
-                        reasons.add(n)
+                self.samples.append((ts, clk, clk_max, {n for n, v in zip(names, parts[6:10])
+                                                        if v.lower() == "active"}))
         try:
             os.remove(self.path)
         except OSError:
             pass
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+
+    def __enter__(self):
+        if not self.enabled:
+            return self
+        try:
+            nv, h = self._nvml_handle()
+            import threading
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h, self.stop), daemon=True)
+            self.thread.start()
+            self.source = f"nvml every {self.period * 1e3:g} ms"
+            return self
+        except Exception:
+            self.thread = None
+        try:
+            self._smi_start()
+            self.source = "nvidia-smi every 200 ms"
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+            self._smi_read()
+
+    def summary(self):
+        if self.source is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        lo, hi = self.t0, self.t1
+        inside = [x for x in self.samples if (lo is None or x[0] >= lo) and (hi is None or x[0] <= hi)]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "source": self.source}
+        reasons = set().union(*(x[3] for x in inside))
+        return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": max(x[2] for x in inside),
+                "reasons": sorted(reasons), "samples": len(inside), "source": self.source}
 
 
 def max_over_ranks(value, device, world):
@@ -255,9 +308,7 @@ def time_step(wl, args, rank, world, device, clocks=True):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    phys = (torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-            else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[torch.cuda.current_device()])
-    with ClockSampler(phys, enabled=clocks) as clk:
+    with ClockSampler(torch.cuda.current_device(), enabled=clocks) as clk:
         clk.mark_start()
         start.record()
         for _ in range(args.steps):
@@ -317,6 +368,9 @@ def time_step(wl, args, rank, world, device, clocks=True):
             "share_of_step": round((q_ms + a_ms) / ms_step, 3),
         },
         "kernels": kernels,
+        "streams": ("W's amax and 2D quantize run on a second stream beside X's amax and ROWCOL quantize; "
+                    "quant_row_sr runs beside gemm_wgrad: per-kernel times are taken on each kernel's own "
+                    "stream, so overlapping shares can sum above 1"),
         "_fprop": (gf["gemm_fprop"], avg_ms["gemm_fprop"], fpeak, fpeak_src),
         "_clocks": clk.summary(),
         "_tensors": (X, W, dY),
@@ -347,6 +401,7 @@ def run_ours(args, rank, world, device):
         "gemm": head["gemm"],
         "quantize": head["quantize"],
         "kernels": head["kernels"],
+        "streams": head["streams"],
         "roofline": {
             "kernel": f"gemm_fp4_pair_kernel<false, false> (fprop, M={T} N={Co} K={Ci}, BF16 out)",
             "bound": "tensor",

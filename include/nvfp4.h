@@ -219,6 +219,12 @@ nvfp4_status nvfp4_mx_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D
  *   column copy) in BF16; amax_rht(dY) -> dY column copy with RHT and SR
  *   (seed); dW = gemm(dY^T q, X^T q) in FP32.
  * Needs T, Cin, Cout multiples of 64.
+ * Both calls run independent branches on a second stream that the library
+ * creates once per device (non-blocking): in the forward, W's amax and 2D
+ * copies beside X's; in the backward, the dY row copy (SR) beside the wgrad
+ * GEMM, whose tensor-pipe work it overlaps.  Each call forks from and joins
+ * back to `stream` with events of its own, so the calls stay stream-ordered
+ * on `stream` (also under stream capture, as a fork/join in the graph).
  */
 size_t nvfp4_linear_workspace_bytes(int64_t T, int64_t Cin, int64_t Cout);
 nvfp4_status nvfp4_linear_fwd(const void* X, const void* W, int64_t T, int64_t Cin, int64_t Cout, void* Y,

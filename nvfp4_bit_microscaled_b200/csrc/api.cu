@@ -116,6 +116,67 @@ nvfp4_status linear_check(int64_t T, int64_t Cin, int64_t Cout, void* ws, size_t
   return NVFP4_OK;
 }
 
+// A second stream of the library's own, one per device, created on first use
+// (non-blocking), and two events per host thread and device, for the linear
+// layer's independent branches.
+nvfp4_status side_stream(int* dev_out, cudaStream_t* out) {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev]) {
+    cudaError_t e = cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  *dev_out = dev;
+  *out = streams[dev];
+  return NVFP4_OK;
+}
+
+// Fork: the side stream starts after the work enqueued on main so far.  Join:
+// main continues after the work enqueued on the side stream since the fork.
+// A stream wait binds to the event's latest record when it is enqueued, so a
+// thread can re-record its two events in every call; calls from several host
+// threads use different events.
+struct Fork {
+  cudaStream_t main = nullptr, side = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+};
+
+nvfp4_status fork(cudaStream_t main, Fork* f) {
+  thread_local cudaEvent_t events[64][2] = {};
+  int dev = 0;
+  nvfp4_status st = side_stream(&dev, &f->side);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < 2 && e == cudaSuccess; ++i)
+    if (!events[dev][i]) e = cudaEventCreateWithFlags(&events[dev][i], cudaEventDisableTiming);
+  if (e != cudaSuccess) return cuda_status(e);
+  f->main = main;
+  f->start = events[dev][0];
+  f->done = events[dev][1];
+  e = cudaEventRecord(f->start, main);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(f->side, f->start, 0);
+  if (e != cudaSuccess) f->side = nullptr;      // nothing was forked
+  return cuda_status(e);
+}
+
+nvfp4_status join(Fork* f) {
+  if (!f->side) return NVFP4_OK;
+  cudaError_t e = cudaEventRecord(f->done, f->side);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(f->main, f->done, 0);
+  f->side = nullptr;
+  return cuda_status(e);
+}
+
+// After an error on one branch: main still waits for what the side stream
+// already holds, so the caller's buffers stay in use until both are done.
+nvfp4_status fail(Fork* f, nvfp4_status st) {
+  (void)join(f);
+  return st;
+}
+
 }  // namespace
 
 namespace nvfp4 {
@@ -131,22 +192,32 @@ nvfp4_status linear_forward(const void* X, const void* W, int64_t T, int64_t Cin
   float* amax = static_cast<float*>(ws);
   const nvfp4_tensor xr = ws_tensor(ws, L, 0), wr = ws_tensor(ws, L, 1), wc = ws_tensor(ws, L, 2);
   nvfp4_status st;
-  // fprop operands: X row-wise (RN), W 2D (RN) with its transposed copy for dgrad
+  // W's amax and 2D copies (RN) on the side stream while X's run on the caller's
+  // stream (without the wgrad operand -- the allocation-free forward -- both run
+  // on the caller's stream: it creates no stream or event)
+  Fork f;
+  cudaStream_t wstream = reinterpret_cast<cudaStream_t>(stream);
+  if (keep_wgrad) {
+    if ((st = fork(wstream, &f)) != NVFP4_OK) return st;
+    wstream = f.side;
+  }
+  nvfp4_stream_t ws_ = reinterpret_cast<nvfp4_stream_t>(wstream);
+  if ((st = nvfp4_amax(W, Cout, Cin, Cin, 0, amax + kAmaxW, ws_)) != NVFP4_OK ||
+      (st = nvfp4_quantize(W, Cout, Cin, Cin, NVFP4_2D, 0, 0, 0, amax + kAmaxW, &wr, &wc, ws_)) != NVFP4_OK)
+    return fail(&f, st);
   // one pass over X gives both its amax (row copy) and its RHT amax (column copy)
-  if ((st = nvfp4_amax(X, T, Cin, Cin, 2, amax + kAmaxX, stream)) != NVFP4_OK) return st;
+  if ((st = nvfp4_amax(X, T, Cin, Cin, 2, amax + kAmaxX, stream)) != NVFP4_OK) return fail(&f, st);
   if (keep_wgrad) {
     // the X row copy (fprop) and the X^T copy with the RHT along tokens, saved
     // for wgrad, from one read of X; amax + kAmaxX holds [max|X|, max|Q X|]
     const nvfp4_tensor xc = ws_tensor(ws, L, 3);
     if ((st = nvfp4_quantize(X, T, Cin, Cin, NVFP4_ROWCOL, 1, 0, 0, amax + kAmaxX, &xr, &xc, stream)) != NVFP4_OK)
-      return st;
+      return fail(&f, st);
+    if ((st = join(&f)) != NVFP4_OK) return st;
   } else if ((st = nvfp4_quantize(X, T, Cin, Cin, NVFP4_ROW, 0, 0, 0, amax + kAmaxX, &xr, nullptr, stream)) !=
              NVFP4_OK) {
     return st;
   }
-  if ((st = nvfp4_amax(W, Cout, Cin, Cin, 0, amax + kAmaxW, stream)) != NVFP4_OK) return st;
-  if ((st = nvfp4_quantize(W, Cout, Cin, Cin, NVFP4_2D, 0, 0, 0, amax + kAmaxW, &wr, &wc, stream)) != NVFP4_OK)
-    return st;
   return nvfp4_gemm(&xr, &wr, Y, NVFP4_OUT_BF16, Cout, stream);
 }
 
@@ -379,18 +450,24 @@ nvfp4_status nvfp4_linear_bwd(const void* dY, int64_t T, int64_t Cin, int64_t Co
   float* amax = static_cast<float*>(workspace);
   const nvfp4_tensor wc = ws_tensor(workspace, L, 2), xc = ws_tensor(workspace, L, 3),
                      gr = ws_tensor(workspace, L, 4), gc = ws_tensor(workspace, L, 5);
-  // dgrad: dX = dY W, dY row-wise with SR, W^T from the 2D column copy
   // one pass over dY gives both its amax (row copy) and its RHT amax (column copy)
   if ((st = nvfp4_amax(dY, T, Cout, Cout, 2, amax + kAmaxDy, stream)) != NVFP4_OK) return st;
-  if ((st = nvfp4_quantize(dY, T, Cout, Cout, NVFP4_ROW, 0, 1, seed, amax + kAmaxDy, &gr, nullptr, stream)) !=
-      NVFP4_OK)
-    return st;
-  if ((st = nvfp4_gemm(&gr, &wc, dX, NVFP4_OUT_BF16, Cin, stream)) != NVFP4_OK) return st;
   // wgrad: dW = dY^T X, both with the RHT along tokens, SR on dY
   if ((st = nvfp4_quantize(dY, T, Cout, Cout, NVFP4_COL, 1, 1, seed, amax + kAmaxDyr, nullptr, &gc, stream)) !=
       NVFP4_OK)
     return st;
-  return nvfp4_gemm(&gc, &xc, dW, NVFP4_OUT_F32, Cin, stream);
+  // the dY row copy (SR) for dgrad on the side stream, next to the wgrad GEMM:
+  // the quantizer is bound by the integer ALU pipe, the GEMM by the tensor pipe,
+  // and its CTAs fit beside the GEMM's on every SM
+  Fork f;
+  if ((st = fork(reinterpret_cast<cudaStream_t>(stream), &f)) != NVFP4_OK) return st;
+  if ((st = nvfp4_gemm(&gc, &xc, dW, NVFP4_OUT_F32, Cin, stream)) != NVFP4_OK ||
+      (st = nvfp4_quantize(dY, T, Cout, Cout, NVFP4_ROW, 0, 1, seed, amax + kAmaxDy, &gr, nullptr,
+                           reinterpret_cast<nvfp4_stream_t>(f.side))) != NVFP4_OK)
+    return fail(&f, st);
+  if ((st = join(&f)) != NVFP4_OK) return st;
+  // dgrad: dX = dY W, dY row-wise with SR, W^T from the 2D column copy
+  return nvfp4_gemm(&gr, &wc, dX, NVFP4_OUT_BF16, Cin, stream);
 }
 
 nvfp4_status nvfp4_read_device_error(unsigned int* code, int clear) {

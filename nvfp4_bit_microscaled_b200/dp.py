@@ -11,6 +11,10 @@ path ("Pretraining Large Language Models with NVFP4", sections 2A and 2B):
   on NCCL it is issued as soon as the wgrad GEMM is done and overlaps the
   dgrad half of the backward pass.
 
+On the GPU the layer also runs independent branches on a second stream: W's
+amax and 2D copies beside X's amax and copies in the forward, and the dY row
+copy (SR) beside the wgrad GEMM in the backward.
+
 Stochastic rounding draws are keyed by the element's index in the whole
 batch (nvfp4_quantize_rows with row0 = rank * T_local), so every rank's
 quantized copies are the matching slices of a one-GPU quantization of the
@@ -61,6 +65,30 @@ class DataParallelLinear:
     def _do(self, kind, fn):
         return self.timer(kind, fn) if self.timer is not None else fn()
 
+    def _side(self, device):
+        """A second CUDA stream of this layer's (None off the GPU)."""
+        if device.type != "cuda":
+            return None
+        if getattr(self, "_side_stream", None) is None:
+            self._side_stream = torch.cuda.Stream(device)
+        return self._side_stream
+
+    def _branch(self, side, fn):
+        """Run fn on the side stream after the work enqueued so far on the
+        current stream; returns the event the current stream must wait for."""
+        if side is None:
+            fn()
+            return None
+        cur = torch.cuda.current_stream()
+        start = torch.cuda.Event()
+        start.record(cur)
+        with torch.cuda.stream(side):
+            side.wait_event(start)
+            fn()
+            done = torch.cuda.Event()
+            done.record(side)
+        return done
+
     def _all_reduce(self, t, op):
         if self.world == 1:
             return
@@ -76,14 +104,18 @@ class DataParallelLinear:
         """Y[T_local, Cout] = X W^T (BF16) for this rank's tokens."""
         assert X.shape == (self.T, self.Cin) and W.shape == (self.Cout, self.Cin)
         d = self._do
+        # W's amax and 2D copies on the side stream while X's are made on this one
+        w_done = self._branch(self._side(X.device), lambda: (
+            d("amax", lambda: api.amax(W, out=self.amax_w)),
+            d("quant_2d", lambda: api.quantize(W, api.TWO_D, self.amax_w, row_out=self.w_row, col_out=self.w_col))))
         d("amax_both", lambda: api.amax(X, rht=2, out=self.amax_x))
         if self.world > 1:
             d("allreduce_amax", lambda: self._all_reduce(self.amax_x, dist.ReduceOp.MAX))
         # X's row copy (fprop) and RHT column copy (wgrad) from one read of X
         d("quant_rowcol_rht", lambda: api.quantize(X, api.ROWCOL, self.amax_x, rht=True, row_out=self.x_row,
                                                    col_out=self.x_col, row0=self.row0))
-        d("amax", lambda: api.amax(W, out=self.amax_w))
-        d("quant_2d", lambda: api.quantize(W, api.TWO_D, self.amax_w, row_out=self.w_row, col_out=self.w_col))
+        if w_done is not None:
+            torch.cuda.current_stream().wait_event(w_done)
         return d("gemm_fprop", lambda: api.gemm(self.x_row, self.w_row, api.OUT_BF16, out=Y))
 
     def backward(self, dY, seed, dX=None, dW=None):
@@ -99,6 +131,11 @@ class DataParallelLinear:
             d("allreduce_amax", lambda: self._all_reduce(self.amax_dy, dist.ReduceOp.MAX))
         d("quant_col_rht_sr", lambda: api.quantize(dY, api.COL, self.amax_dy[1:2], rht=True, sr=True, seed=seed,
                                                    col_out=self.dy_col, row0=self.row0))
+        side = self._side(dY.device)
+        start = None
+        if side is not None:
+            start = torch.cuda.Event()
+            start.record(torch.cuda.current_stream())
         dW = d("gemm_wgrad", lambda: api.gemm(self.dy_col, self.x_col, api.OUT_F32, out=dW))
         pending = None
         if self.world > 1:
@@ -106,8 +143,19 @@ class DataParallelLinear:
                 pending = dist.all_reduce(dW, op=dist.ReduceOp.SUM, group=self.group, async_op=True)
             else:
                 d("allreduce_dw", lambda: self._all_reduce(dW, dist.ReduceOp.SUM))
-        d("quant_row_sr", lambda: api.quantize(dY, api.ROW, self.amax_dy[0:1], sr=True, seed=seed,
-                                               row_out=self.dy_row, row0=self.row0))
+        # the dY row copy (SR) on the side stream, next to the wgrad GEMM: the
+        # quantizer is bound by the integer ALU pipe, the GEMM by the tensor pipe
+        row_sr = lambda: d("quant_row_sr", lambda: api.quantize(dY, api.ROW, self.amax_dy[0:1], sr=True, seed=seed,
+                                                                row_out=self.dy_row, row0=self.row0))
+        if side is None:
+            row_sr()
+        else:
+            with torch.cuda.stream(side):
+                side.wait_event(start)
+                row_sr()
+                done = torch.cuda.Event()
+                done.record(side)
+            torch.cuda.current_stream().wait_event(done)
         dX = d("gemm_dgrad", lambda: api.gemm(self.dy_row, self.w_col, api.OUT_BF16, out=dX))
         if pending is not None:
             d("allreduce_dw_wait", pending.wait)   # the current stream waits for the all-reduce

@@ -8,6 +8,7 @@ import hashlib
 import json
 import os
 import re
+import time
 
 import bench
 
@@ -17,19 +18,26 @@ def _line(ts, sm, reasons=("Not Active",) * 4):
     return ", ".join([stamp, "0", str(sm), "1965", "990.0", "0x0000000000000004", *reasons]) + "\n"
 
 
-def test_clock_summary_keeps_timed_samples_and_reasons(tmp_path):
+def _smi_sampler(tmp_path, lines):
     c = bench.ClockSampler(0)
     c.path = str(tmp_path / "clocks.csv")
-    c.proc = object()                          # as if nvidia-smi had been started
-    t0 = 1_800_000_000.0
-    c.t0, c.t1 = t0, t0 + 10.0
+    c.source = "nvidia-smi every 200 ms"
     with open(c.path, "w") as f:
-        f.write(_line(t0 - 5.0, 600, ("Active",) * 4))                 # before the timed region
-        f.write(_line(t0 + 1.0, 1700))
-        f.write(_line(t0 + 2.0, 1650, ("Not Active", "Not Active", "Not Active", "Active")))
-        f.write(_line(t0 + 3.0, 1750))
-        f.write("garbage line\n")
-        f.write(_line(t0 + 20.0, 300, ("Active",) * 4))                # after it
+        f.writelines(lines)
+    c._smi_read()
+    return c
+
+
+def test_clock_summary_keeps_timed_samples_and_reasons(tmp_path):
+    t0 = 1_800_000_000.0
+    c = _smi_sampler(tmp_path, [
+        _line(t0 - 5.0, 600, ("Active",) * 4),                 # before the timed region
+        _line(t0 + 1.0, 1700),
+        _line(t0 + 2.0, 1650, ("Not Active", "Not Active", "Not Active", "Active")),
+        _line(t0 + 3.0, 1750),
+        "garbage line\n",
+        _line(t0 + 20.0, 300, ("Active",) * 4)])               # after it
+    c.t0, c.t1 = t0, t0 + 10.0
     s = c.summary()
     assert s["samples"] == 3 and s["sm_mhz"] == 1700 and s["sm_max_mhz"] == 1965
     assert s["reasons"] == ["sw_power_cap"]
@@ -37,24 +45,59 @@ def test_clock_summary_keeps_timed_samples_and_reasons(tmp_path):
 
 
 def test_clock_summary_flags_hardware_slowdown(tmp_path):
-    c = bench.ClockSampler(0)
-    c.path = str(tmp_path / "clocks.csv")
-    c.proc = object()
     t0 = 1_800_000_000.0
+    c = _smi_sampler(tmp_path, [_line(t0 + 1.0, 1200, ("Active", "Not Active", "Active", "Not Active"))])
     c.t0, c.t1 = t0, t0 + 10.0
-    with open(c.path, "w") as f:
-        f.write(_line(t0 + 1.0, 1200, ("Active", "Not Active", "Active", "Not Active")))
-    s = c.summary()
-    assert s["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert c.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
 
 
 def test_clock_summary_without_samples(tmp_path):
     c = bench.ClockSampler(0)
-    assert c.summary()["reasons"] == ["nvidia-smi unavailable"]
-    c.path = str(tmp_path / "empty.csv")
-    c.proc = object()
-    open(c.path, "w").close()
+    assert c.summary()["reasons"] == ["clock sampling unavailable"]
+    c = _smi_sampler(tmp_path, [])
     assert c.summary()["reasons"] == ["no samples"]
+
+
+class _FakeNvml:
+    """Clock queries of a fake NVML: a clock sequence and one reason bit mask."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonSwPowerCap = 0x4
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+
+    def __init__(self, clocks, reasons):
+        self.clocks, self.reasons, self.calls = list(clocks), reasons, 0
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        self.calls += 1
+        return self.clocks[min(self.calls - 1, len(self.clocks) - 1)]
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.reasons
+
+
+def test_nvml_sampler_decodes_reason_bits():
+    import threading
+    nv = _FakeNvml([1500, 1520, 1480], 0x4 | 0x1)            # power cap (+ the idle bit, not reported)
+    c = bench.ClockSampler(0, period_s=0.001)
+    c.source = "nvml"
+    stop = threading.Event()
+    th = threading.Thread(target=c._nvml_loop, args=(nv, None, stop))
+    c.mark_start()
+    th.start()
+    deadline = time.time() + 10.0
+    while nv.calls < 5 and time.time() < deadline:
+        time.sleep(0.001)
+    stop.set()
+    th.join()
+    c.mark_end()
+    s = c.summary()
+    assert s["sm_max_mhz"] == 1965 and s["samples"] >= 3
+    assert s["reasons"] == ["sw_power_cap"] and s["sm_mhz"] in (1480, 1500, 1520)
 
 
 def test_gemm_profile_is_reported_only_for_the_profiled_source(tmp_path, monkeypatch):
