@@ -205,34 +205,30 @@ __device__ __forceinline__ u32x4 sr_words(uint64_t g, uint32_t domain, uint32_t 
 // ("Pretraining Large Language Models with NVFP4", section 2B.4 and the
 // "De Gok" example: 3.4 goes to 4 with probability 0.4.)
 //
-// |y| >= 1: the E2M1 grid is the FP32 values with one mantissa bit, so p is
-// the 22 bits below it over 2^22, and u < p  <=>  (w >> 10) < frac22  <=>
-// frac22 + ((~w) >> 10) carries into that bit: add and truncate, on the
-// signed bit pattern (the carry never reaches the sign bit and the mask keeps
-// it).  (~w) >> 10 == (2^22 - 1) - (w >> 10): one three-input add.  It also
-// runs without the saturation at 6: a value in (6, 6.4] (the E4M3 block scale
-// rounds to nearest, so |y| stays below 6.4) comes out as 6 or 8, and the
-// saturating E2M1 conversion turns both into 6, the code the saturated value
-// gives.
-//
-// |y| < 1: the grid is {0, 0.5, 1}, a lattice of step 0.5, and the rule is
-// q = ceil_0.5(|y| - u/2) exactly (round up iff p > u).  It is evaluated in
-// FP32 with upward rounding: z = RU(|y| - 2^-25 (w >> 8)) is one fma, and
-// ceil_0.5(RU(x)) = ceil_0.5(x) for every real x because the lattice points
-// are floats; RU(z + 1.5 * 2^22) - 1.5 * 2^22 then takes the ceiling on the
-// lattice (z + 1.5 * 2^22 lies in a binade whose ulp is 0.5).  Exact for every
-// |y| < 1, tiny values included, with no integer work: the rounding runs on
-// the FMA pipe, which these kernels leave idle, instead of the integer ALU
-// pipe they are bound by.
-//
-// Both are the same decision as the definition above, bit for bit.
+// One formula for the whole range.  The grid step at |y| is s = 0.5 below 2
+// and half the power of two of |y|'s binade above (1 in [2, 4), 2 in
+// [4, 8)): s = 2^floor(log2 max(|y|, 1)) / 2, taken from the exponent bits.
+// With |y| = lo + p*s, rounding up iff u < p is q = ceil_s(|y| - u*s): the
+// argument lies in (lo, lo + s) exactly when u < p and in (lo - s, lo]
+// otherwise, and below a binade boundary the finer lattice of the lower
+// binade still has lo as a point.  u*s is exact (a 24-bit integer times a
+// power of two), so z = RU(|y| - u*s) is one fma with upward rounding, and
+// ceil_s(RU(x)) = ceil_s(x) because the lattice points are floats.  Then
+// RU(z + M) - M with M = 1.5 * 2^23 * s takes the ceiling on the lattice
+// (z + M lies in a binade whose ulp is s).  A value in (6, 6.4] (the E4M3
+// block scale rounds to nearest, so |y| stays below 6.4) comes out as 6 or 8,
+// and the saturating E2M1 conversion turns both into 6, the code the
+// saturated value gives.  The same decision as the definition above, bit for
+// bit; a CPU emulation with directed rounding agreed with it on every float
+// in [0, 6.4).  Four integer-ALU operations per element (the shift of w, the
+// max, the exponent mask, the sign), the rest on the FMA pipe.
 __device__ __forceinline__ float sr_magnitude(float y, uint32_t w) {
-  const uint32_t b = __float_as_uint(y);
-  const float upper = __uint_as_float((b + 0x003FFFFFu - (w >> 10)) & ~0x003FFFFFu);
-  const float z = __fmaf_ru(-2.98023223876953125e-08f, __uint2float_rn(w >> 8), fabsf(y));  // -2^-25
-  const float q = __fsub_rn(__fadd_ru(z, 6291456.0f), 6291456.0f);                            // 1.5 * 2^22
-  const float lower = __uint_as_float(__float_as_uint(q) | (b & 0x80000000u));
-  return fabsf(y) >= 1.0f ? upper : lower;
+  const float a = fabsf(y);
+  const float s = __fmul_rn(__uint_as_float(__float_as_uint(fmaxf(a, 1.0f)) & 0x7F800000u), 0.5f);
+  const float z = __fmaf_ru(-__uint2float_rn(w >> 8), __fmul_rn(s, 5.9604644775390625e-08f), a);  // 2^-24
+  const float m = __fmul_rn(s, 12582912.0f);                                                        // 1.5 * 2^23
+  const float q = __fsub_rn(__fadd_ru(z, m), m);
+  return __uint_as_float(__float_as_uint(q) | (__float_as_uint(y) & 0x80000000u));
 }
 
 // --------------------------------------------------------------------------
