@@ -247,6 +247,35 @@ class EventTimer:
         return out
 
 
+class AloneTimer:
+    """timer(kind, fn) that times each library call alone, after the step's
+    timed region: the device is idle before every launch (so no kernel of the
+    other stream runs beside it), L2 is flushed with a 256 MB write, and the
+    call is launched `reps` times; collectives run once, untimed."""
+
+    def __init__(self, device, reps=5):
+        self.reps = reps
+        self.ms = {}
+        self.scratch = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def __call__(self, kind, fn):
+        if kind.startswith("allreduce"):
+            return fn()
+        times = []
+        out = None
+        for _ in range(self.reps):
+            torch.cuda.synchronize()
+            self.scratch.fill_(1)
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            out = fn()
+            e.record()
+            torch.cuda.synchronize()
+            times.append(s.elapsed_time(e))
+        self.ms.setdefault(kind, []).append(sum(times) / len(times))
+        return out
+
+
 KERNELS_PER_STEP = 10  # 3 amax + 4 quantize + 3 GEMM kernels (no scale padding at these shapes)
 QUANT_KINDS = ("quant_rowcol_rht", "quant_2d", "quant_row_sr", "quant_col_rht_sr")
 
@@ -323,6 +352,16 @@ def time_step(wl, args, rank, world, device, clocks=True):
     if err:
         raise RuntimeError(f"device error word {err} after the timed region")
 
+    # every kernel once more, alone (outside the timed region; the step above is the number)
+    alone = AloneTimer(device)
+    layer.timer = alone
+    step()
+    torch.cuda.synchronize()
+    layer.timer = timer
+    err = api.read_device_error(clear=True)
+    if err:
+        raise RuntimeError(f"device error word {err} after the isolated timings")
+
     per_kind = {}
     for kind, s, e in timer.events:
         per_kind.setdefault(kind, []).append(s.elapsed_time(e))
@@ -350,6 +389,17 @@ def time_step(wl, args, rank, world, device, clocks=True):
             entry["gbs"] = round(kb[k] / n / (avg_ms[k] * 1e-3) / 1e9, 1)
             entry["frac_hbm"] = round(entry["gbs"] / hbm, 4)
         kernels[k] = entry
+    kernels_alone = {}
+    for k, v in alone.ms.items():
+        ms = sum(v) / len(v)
+        entry = {"ms_per_launch": round(ms, 4)}
+        if k in gf:
+            entry["tflops"] = round(gf[k] / (ms * 1e-3) / 1e12, 1)
+            entry["frac_fp4_peak"] = round(entry["tflops"] / fpeak, 4)
+        elif k in kb:
+            entry["gbs"] = round(kb[k] / len(v) / (ms * 1e-3) / 1e9, 1)
+            entry["frac_hbm"] = round(entry["gbs"] / hbm, 4)
+        kernels_alone[k] = entry
     return {
         "workload": wl["desc"],
         "ms_per_step": round(ms_step, 4),
@@ -371,6 +421,10 @@ def time_step(wl, args, rank, world, device, clocks=True):
         "streams": ("W's amax and 2D quantize run on a second stream beside X's amax and ROWCOL quantize; "
                     "quant_row_sr runs beside gemm_wgrad: per-kernel times are taken on each kernel's own "
                     "stream, so overlapping shares can sum above 1"),
+        "kernels_alone": kernels_alone,
+        "kernels_alone_note": ("each call once more after the timed region, alone on an idle device, L2 "
+                               "flushed before each of 5 launches: the kernel's own rate, without the "
+                               "second stream's overlap"),
         "_fprop": (gf["gemm_fprop"], avg_ms["gemm_fprop"], fpeak, fpeak_src),
         "_clocks": clk.summary(),
         "_tensors": (X, W, dY),
@@ -402,6 +456,8 @@ def run_ours(args, rank, world, device):
         "quantize": head["quantize"],
         "kernels": head["kernels"],
         "streams": head["streams"],
+        "kernels_alone": head["kernels_alone"],
+        "kernels_alone_note": head["kernels_alone_note"],
         "roofline": {
             "kernel": f"gemm_fp4_pair_kernel<false, false> (fprop, M={T} N={Co} K={Ci}, BF16 out)",
             "bound": "tensor",

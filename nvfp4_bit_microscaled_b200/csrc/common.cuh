@@ -199,6 +199,87 @@ __device__ __forceinline__ u32x4 sr_words(uint64_t g, uint32_t domain, uint32_t 
                        k0, k1);
 }
 
+// --------------------------------------------------------------------------
+// Packed FP32 pairs (one instruction for two lanes of arithmetic; CUDA's
+// headers provide the round-to-nearest forms, these add the directed ones)
+// --------------------------------------------------------------------------
+__device__ __forceinline__ float2 ffma2_ru(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rp.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2_ru(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rp.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fsub2_rn(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// Two BF16 values (low and high half of w) as an FP32 pair.
+__device__ __forceinline__ float2 bf16x2_to_f32x2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// max(|a|, |b|, |c|) in one instruction.
+__device__ __forceinline__ float max3_abs(float a, float b, float c) {
+  float d;
+  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// max |v_i| over the 16 first (Y = false) or second (Y = true) components.
+template <bool Y>
+__device__ __forceinline__ float absmax16(const float2 (&v)[16]) {
+  auto c = [&](int i) { return Y ? v[i].y : v[i].x; };
+  float m = max3_abs(c(0), c(1), c(2));
+#pragma unroll
+  for (int i = 3; i < 15; i += 2) m = max3_abs(m, c(i), c(i + 1));
+  return max3_abs(m, c(15), 0.0f);
+}
+
+// The 16-point RHT butterflies of two channels at once (v[i] = element i of
+// both), the same stages, order and FP32 roundings as fwht16_absmax<true>
+// (h = 1, 2, 4, 8), with the random signs s_i kept symbolically: on return
+// neg[i] says that the true value of element i is -v[i].  A butterfly of
+// a = sa*va and b = sb*vb is (sa*(va + vb), sa*(va - vb)) when sa == sb and
+// (sa*(va - vb), sa*(va + vb)) otherwise; round-to-nearest is symmetric, so
+// the registers hold the true results up to those signs, bit for bit.  After
+// unrolling the signs are compile-time constants.
+__device__ __forceinline__ void fwht16_x2(float2 (&v)[16], bool (&neg)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) neg[i] = rht_negates(i);
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if ((j & h) == 0) {
+        const float2 a = v[j], b = v[j + h];
+        const float2 sum = __fadd2_rn(a, b), dif = fsub2_rn(a, b);
+        const bool same = neg[j] == neg[j + h];
+        v[j] = same ? sum : dif;
+        v[j + h] = same ? dif : sum;
+        neg[j + h] = neg[j];
+      }
+    }
+  }
+}
+
 // Stochastic rounding of a scaled value to the E2M1 grid: between the two
 // neighbouring grid magnitudes lo and lo + step, round up iff the 24-bit
 // uniform u = (w >> 8) * 2^-24 is below the fractional position p.
@@ -222,13 +303,24 @@ __device__ __forceinline__ u32x4 sr_words(uint64_t g, uint32_t domain, uint32_t 
 // bit; a CPU emulation with directed rounding agreed with it on every float
 // in [0, 6.4).  Four integer-ALU operations per element (the shift of w, the
 // max, the exponent mask, the sign), the rest on the FMA pipe.
-__device__ __forceinline__ float sr_magnitude(float y, uint32_t w) {
-  const float a = fabsf(y);
-  const float s = __fmul_rn(__uint_as_float(__float_as_uint(fmaxf(a, 1.0f)) & 0x7F800000u), 0.5f);
-  const float z = __fmaf_ru(-__uint2float_rn(w >> 8), __fmul_rn(s, 5.9604644775390625e-08f), a);  // 2^-24
-  const float m = __fmul_rn(s, 12582912.0f);                                                        // 1.5 * 2^23
-  const float q = __fsub_rn(__fadd_ru(z, m), m);
-  return __uint_as_float(__float_as_uint(q) | (__float_as_uint(y) & 0x80000000u));
+//
+// Two elements at a time (y.x with word w0, y.y with w1).  With FLIP the
+// result's sign is the opposite of y's (the caller's register holds -y, as
+// fwht16_x2 leaves it).
+template <bool FLIP>
+__device__ __forceinline__ float2 sr_magnitude2(float2 y, uint32_t w0, uint32_t w1) {
+  const float2 a = make_float2(fabsf(y.x), fabsf(y.y));
+  // 2s: the power of two of max(|y|, 1)'s binade
+  const float2 s2 = make_float2(__uint_as_float(__float_as_uint(fmaxf(a.x, 1.0f)) & 0x7F800000u),
+                                __uint_as_float(__float_as_uint(fmaxf(a.y, 1.0f)) & 0x7F800000u));
+  const float2 k = make_float2(__uint2float_rn(w0 >> 8), __uint2float_rn(w1 >> 8));
+  const float2 z = ffma2_ru(k, __fmul2_rn(s2, make_float2(-2.98023223876953125e-08f, -2.98023223876953125e-08f)),
+                            a);                                                           // |y| - u*s, u*s = k*2s*2^-25
+  const float2 m = __fmul2_rn(s2, make_float2(6291456.0f, 6291456.0f));                   // 1.5*2^23*s
+  const float2 q = fsub2_rn(fadd2_ru(z, m), m);
+  const uint32_t sx = __float_as_uint(y.x) & 0x80000000u, sy = __float_as_uint(y.y) & 0x80000000u;
+  return make_float2(__uint_as_float(__float_as_uint(q.x) | (FLIP ? sx ^ 0x80000000u : sx)),
+                     __uint_as_float(__float_as_uint(q.y) | (FLIP ? sy ^ 0x80000000u : sy)));
 }
 
 // --------------------------------------------------------------------------

@@ -117,27 +117,43 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (base + u * nwarps >= items) break;  // warp-uniform
-      const uint32_t mb = max(absmax_bits8(v[u][0]), absmax_bits8(v[u][1]));
-      const BlockScale bs = block_scale_t(bf16_bits_to_f32(mb), s_enc, r_tbl);
-      float y[16];
-      unpack8(v[u][0], y);
-      unpack8(v[u][1], y + 8);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(y[i], bs.r);
+      uint32_t sfb;
+      uint32_t w0, w1;
       if (SR) {
+        // elements (2k, 2k+1) as FP32 pairs: the scaling and the SR decision run packed
+        const uint4 a = v[u][0], b = v[u][1];
+        float2 y[8] = {bf16x2_to_f32x2(a.x), bf16x2_to_f32x2(a.y), bf16x2_to_f32x2(a.z), bf16x2_to_f32x2(a.w),
+                       bf16x2_to_f32x2(b.x), bf16x2_to_f32x2(b.y), bf16x2_to_f32x2(b.z), bf16x2_to_f32x2(b.w)};
+        float m = max3_abs(y[0].x, y[0].y, y[1].x);
+#pragma unroll
+        for (int k = 1; k < 7; ++k) m = max3_abs(m, y[k].y, y[k + 1].x);
+        m = max3_abs(m, y[7].y, 0.0f);
+        const BlockScale bs0 = block_scale_t(m, s_enc, r_tbl);
+        sfb = bs0.sf;
+        const float2 r2 = make_float2(bs0.r, bs0.r);
         const uint64_t g = static_cast<uint64_t>(rr[u] * C + bb[u] * 16 + idx0) >> 2;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const u32x4 w = sr_words<NARROW>(g + q, kDomainRowSR, k0, k1);
-          y[4 * q + 0] = sr_magnitude(y[4 * q + 0], w.x);
-          y[4 * q + 1] = sr_magnitude(y[4 * q + 1], w.y);
-          y[4 * q + 2] = sr_magnitude(y[4 * q + 2], w.z);
-          y[4 * q + 3] = sr_magnitude(y[4 * q + 3], w.w);
+          y[2 * q] = sr_magnitude2<false>(__fmul2_rn(y[2 * q], r2), w.x, w.y);
+          y[2 * q + 1] = sr_magnitude2<false>(__fmul2_rn(y[2 * q + 1], r2), w.z, w.w);
         }
+        w0 = clear_negative_zero(f32x8_to_e2m1x8(y[0].x, y[0].y, y[1].x, y[1].y, y[2].x, y[2].y, y[3].x, y[3].y));
+        w1 = clear_negative_zero(f32x8_to_e2m1x8(y[4].x, y[4].y, y[5].x, y[5].y, y[6].x, y[6].y, y[7].x, y[7].y));
+      } else {
+        const uint32_t mb = max(absmax_bits8(v[u][0]), absmax_bits8(v[u][1]));
+        const BlockScale bs0 = block_scale_t(bf16_bits_to_f32(mb), s_enc, r_tbl);
+        sfb = bs0.sf;
+        float y[16];
+        unpack8(v[u][0], y);
+        unpack8(v[u][1], y + 8);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(y[i], bs0.r);
+        w0 = pack8(y);
+        w1 = pack8(y + 8);
       }
-      const uint32_t w0 = pack8(y), w1 = pack8(y + 8);
       if (ok[u]) *reinterpret_cast<uint2*>(data + rr[u] * half_c + bb[u] * 8) = make_uint2(w0, w1);
-      uint32_t word = ok[u] ? (bs.sf << (8 * (lane & 3))) : 0u;
+      uint32_t word = ok[u] ? (sfb << (8 * (lane & 3))) : 0u;
       word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
       word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
       if ((lane & 3) == 0 && ok[u]) *reinterpret_cast<uint32_t*>(sf + sf_offset(rr[u], bb[u], sp)) = word;
@@ -196,59 +212,78 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
       // SR counter of (tbase, c0): its element index in the whole tensor / 4
       // (C, c0 and idx0 are multiples of 4, so row i adds i * C/4 exactly)
       const uint64_t gq = static_cast<uint64_t>(tbase * C + c0 + idx0) >> 2;
-      float v[4][16];
+      // v[p][i]: channels c0 + 2p (first) and c0 + 2p + 1 (second) at token tbase + i,
+      // as FP32 pairs, so the transform and the scaling run as packed instructions
+      float2 v[2][16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const uint2 raw = __ldcs(reinterpret_cast<const uint2*>(x + (tbase + i) * ld + c0));
-        v[0][i] = __uint_as_float(raw.x << 16);
-        v[1][i] = __uint_as_float(raw.x & 0xFFFF0000u);
-        v[2][i] = __uint_as_float(raw.y << 16);
-        v[3][i] = __uint_as_float(raw.y & 0xFFFF0000u);
-        if (RHT && rht_negates(i)) {  // s_i x_i: a negation the first butterfly's adds absorb
+        v[0][i] = bf16x2_to_f32x2(raw.x);
+        v[1][i] = bf16x2_to_f32x2(raw.y);
+      }
+      bool neg[16];   // true value of element i = -register (the RHT's signs, tracked at compile time)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) v[c][i] = -v[c][i];
-        }
+      for (int i = 0; i < 16; ++i) neg[i] = false;
+      float m[4];
+      if (RHT) {
+        bool neg1[16];
+        fwht16_x2(v[0], neg);
+        fwht16_x2(v[1], neg1);   // the same compile-time signs
+        // the 1/4 commutes with the maximum (exact power of two, monotone)
+        m[0] = __fmul_rn(absmax16<false>(v[0]), 0.25f);
+        m[1] = __fmul_rn(absmax16<true>(v[0]), 0.25f);
+        m[2] = __fmul_rn(absmax16<false>(v[1]), 0.25f);
+        m[3] = __fmul_rn(absmax16<true>(v[1]), 0.25f);
+        const float2 q4 = make_float2(0.25f, 0.25f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[0][i] = __fmul2_rn(v[0][i], q4), v[1][i] = __fmul2_rn(v[1][i], q4);
+      } else {
+        m[0] = absmax16<false>(v[0]);
+        m[1] = absmax16<true>(v[0]);
+        m[2] = absmax16<false>(v[1]);
+        m[3] = absmax16<true>(v[1]);
       }
       float r[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        float m = 0.0f;
-        if (RHT) {
-          // max |v| of the transformed run from the last butterfly's inputs;
-          // the 1/4 commutes with the maximum (exact power of two, monotone)
-          m = __fmul_rn(fwht16_absmax<true>(v[c]), 0.25f);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) v[c][i] = __fmul_rn(v[c][i], 0.25f);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[c][i]));
-        }
-        const BlockScale bs = block_scale_t(m, s_enc, r_tbl);
+        const BlockScale bs = block_scale_t(m[c], s_enc, r_tbl);
         r[c] = bs.r;
         sfw[c] |= bs.sf << (8 * tb);
       }
+      const float2 r0 = make_float2(r[0], r[1]), r1 = make_float2(r[2], r[3]);
 #pragma unroll
-      for (int i = 0; i < 16; i += 2) {
-        float y0[4], y1[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          y0[c] = __fmul_rn(v[c][i], r[c]);
-          y1[c] = __fmul_rn(v[c][i + 1], r[c]);
-        }
+      for (int i = 0; i < 16; ++i) {
         if (SR) {
-          const u32x4 wa = sr_words<NARROW>(gq + i * cq, kDomainColSR, k0, k1);
-          const u32x4 wb = sr_words<NARROW>(gq + (i + 1) * cq, kDomainColSR, k0, k1);
-          y0[0] = sr_magnitude(y0[0], wa.x); y0[1] = sr_magnitude(y0[1], wa.y);
-          y0[2] = sr_magnitude(y0[2], wa.z); y0[3] = sr_magnitude(y0[3], wa.w);
-          y1[0] = sr_magnitude(y1[0], wb.x); y1[1] = sr_magnitude(y1[1], wb.y);
-          y1[2] = sr_magnitude(y1[2], wb.z); y1[3] = sr_magnitude(y1[3], wb.w);
+          // y = v * r, then the SR decision on |y| with the true sign (register sign, flipped by neg[i])
+          const float2 y0 = __fmul2_rn(v[0][i], r0), y1 = __fmul2_rn(v[1][i], r1);
+          const u32x4 w = sr_words<NARROW>(gq + i * cq, kDomainColSR, k0, k1);
+          if (neg[i]) {
+            v[0][i] = sr_magnitude2<true>(y0, w.x, w.y);
+            v[1][i] = sr_magnitude2<true>(y1, w.z, w.w);
+          } else {
+            v[0][i] = sr_magnitude2<false>(y0, w.x, w.y);
+            v[1][i] = sr_magnitude2<false>(y1, w.z, w.w);
+          }
+        } else {
+          const float2 rn0 = make_float2(-r[0], -r[1]), rn1 = make_float2(-r[2], -r[3]);
+          v[0][i] = __fmul2_rn(v[0][i], neg[i] ? rn0 : r0);
+          v[1][i] = __fmul2_rn(v[1][i], neg[i] ? rn1 : r1);
         }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) v[c][i] = y0[c], v[c][i + 1] = y1[c];  // scaled values replace the inputs
       }
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        reinterpret_cast<uint2*>(data + (c0 + c) * half_r + t0 / 2)[tb] = make_uint2(pack8(v[c]), pack8(v[c] + 8));
+      for (int p = 0; p < 2; ++p) {
+        const float2* w = v[p];
+        const uint32_t a0 = clear_negative_zero(
+            f32x8_to_e2m1x8(w[0].x, w[1].x, w[2].x, w[3].x, w[4].x, w[5].x, w[6].x, w[7].x));
+        const uint32_t a1 = clear_negative_zero(
+            f32x8_to_e2m1x8(w[8].x, w[9].x, w[10].x, w[11].x, w[12].x, w[13].x, w[14].x, w[15].x));
+        const uint32_t b0 = clear_negative_zero(
+            f32x8_to_e2m1x8(w[0].y, w[1].y, w[2].y, w[3].y, w[4].y, w[5].y, w[6].y, w[7].y));
+        const uint32_t b1 = clear_negative_zero(
+            f32x8_to_e2m1x8(w[8].y, w[9].y, w[10].y, w[11].y, w[12].y, w[13].y, w[14].y, w[15].y));
+        reinterpret_cast<uint2*>(data + (c0 + 2 * p) * half_r + t0 / 2)[tb] = make_uint2(a0, a1);
+        reinterpret_cast<uint2*>(data + (c0 + 2 * p + 1) * half_r + t0 / 2)[tb] = make_uint2(b0, b1);
+      }
     }
 #pragma unroll
     for (int c = 0; c < 4; ++c) *reinterpret_cast<uint32_t*>(sf + sf_offset(c0 + c, 4 * q, sp)) = sfw[c];

@@ -1,10 +1,10 @@
-/* CPU check of the kernels' stochastic-rounding decision (sr_magnitude in
+/* CPU check of the kernels' stochastic-rounding decision (sr_magnitude2 in
  * csrc/common.cuh) against the rule it implements: between the neighbouring
  * E2M1 grid magnitudes lo and hi, round up iff u = (w >> 8) * 2^-24 is below
  * (|y| - lo) / (hi - lo)  ("Pretraining Large Language Models with NVFP4",
- * section 2B.4).  The kernel's arithmetic is restated here with C99 directed
- * rounding (the GPU's __fmaf_ru / __fadd_ru); the rule is evaluated exactly in
- * double.  Usage: sr_decision_check STRIDE -- every STRIDE-th float in
+ * section 2B.4).  The kernel's arithmetic is restated here one element at a
+ * time, with C99 directed rounding for the GPU's fma.rp / add.rp on FP32
+ * pairs; the rule is evaluated exactly in double.  Usage: sr_decision_check STRIDE -- every STRIDE-th float in
  * [0, 6.4) (both signs alternate) with two words each: a fixed corner word
  * and a pseudo-random one.  Prints the count of mismatches; exit 1 if any. */
 #include <fenv.h>
@@ -32,15 +32,15 @@ static float add_ru(float a, float b) {
   return r;
 }
 
-/* the kernel's formula: lattice step s from |y|'s binade (0.5 below 2), then
- * ceil_s(RU(|y| - u*s)) by the magic-number add, sign restored */
+/* the kernel's formula: 2s, twice the lattice step, from |y|'s binade (s = 0.5
+ * below 2), then ceil_s(RU(|y| - u*s)) by the magic-number add, sign restored */
 static float kernel_decision(float y, uint32_t w) {
   const float a = fabsf(y);
-  volatile float s = u2f(f2u(fmaxf(a, 1.0f)) & 0x7F800000u) * 0.5f;
+  volatile float s2 = u2f(f2u(fmaxf(a, 1.0f)) & 0x7F800000u);
   volatile float k = (float)(w >> 8);
-  volatile float st = s * 5.9604644775390625e-08f;
-  const float z = fma_ru(-k, st, a);
-  volatile float m = s * 12582912.0f;
+  volatile float st = s2 * -2.98023223876953125e-08f;   /* -s * 2^-24 */
+  const float z = fma_ru(k, st, a);
+  volatile float m = s2 * 6291456.0f;                    /* 1.5 * 2^23 * s */
   volatile float t = add_ru(z, m);
   const float q = t - m;
   return u2f(f2u(q) | (f2u(y) & 0x80000000u));
