@@ -431,6 +431,19 @@ __global__ void __launch_bounds__(256, 2) quant_rowcol_kernel(
 #pragma unroll
       for (int i = 0; i < 16; ++i)
         raw[i] = lane_ok ? __ldcs(reinterpret_cast<const uint2*>(x + (tbase + i) * ld + c0)) : make_uint2(0u, 0u);
+      {
+        // the warp's next band into L2 while this one is computed: lane l takes
+        // row l % 16, 128-byte half l / 16 (the next band of this item, else the
+        // first band of the warp's next item)
+        int64_t nt = tbase + 16, ncw = cw;
+        if (tb + 1 >= nb) {
+          const int64_t nit = it + nwarps, nq = nit / ng;
+          nt = nit < items ? nq * 64 : -1;
+          ncw = (nit - nq * ng) * 128;
+        }
+        const int64_t pc = ncw + 64 * (lane >> 4);
+        if (nt >= 0 && pc < C) prefetch_l2(x + (nt + (lane & 15)) * ld + pc);
+      }
 #pragma unroll
       for (int i = 0; i < 16; ++i) *reinterpret_cast<uint2*>(&bw[i][8 * lane]) = raw[i];
       if (!flag_col && lane_ok) {
