@@ -75,15 +75,15 @@ __global__ void __launch_bounds__(256) amax_rows_kernel(const uint16_t* __restri
 // 16-row band x 4 consecutive columns: sixteen 8-byte loads, coalesced along
 // the row across the warp (256 bytes per row per warp).  The 1/4 is applied
 // after the maximum (an exact power-of-two scale commutes with max), and the
-// transform's last butterfly stage is folded into the maximum
-// (fwht16_absmax).
+// transform's last butterfly stage is folded into the maximum.  The first
+// three stages run on FP32 pairs of columns (fwht16_x2).
 // Non-finite inputs: every thread also keeps the BF16 magnitude maximum of
 // what it read; a NaN or infinity there (bits >= 0x7F80) makes its RHT
 // maximum NaN, and the reduction runs on float bit patterns, where the NaN
 // 0x7FC00000 orders above every finite value and infinity, so the result is
 // NaN exactly when the tensor holds a non-finite element.
 template <bool BOTH>
-__global__ void __launch_bounds__(256, 3) amax_rht_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+__global__ void __launch_bounds__(256, 2) amax_rht_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
                                                             int64_t ld, unsigned int* __restrict__ out) {
   const int64_t groups = C / 4;
   const int64_t items = (R / 16) * groups;
@@ -107,15 +107,20 @@ __global__ void __launch_bounds__(256, 3) amax_rht_kernel(const uint16_t* __rest
     for (int i = 0; i < 16; ++i)
       mplain = __vmaxu2(mplain, __vmaxu2(v[i].x & 0x7FFF7FFFu, v[i].y & 0x7FFF7FFFu));
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float f[16];
+    for (int p = 0; p < 2; ++p) {   // channels 2p, 2p + 1 as FP32 pairs
+      float2 f[16];
+      bool neg[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint32_t word = (c < 2) ? v[i].x : v[i].y;
-        const float xi = __uint_as_float((c & 1) ? (word & 0xFFFF0000u) : (word << 16));
-        f[i] = rht_negates(i) ? -xi : xi;  // s_i x_i
-      }
-      m = fmaxf(m, fwht16_absmax<false>(f));
+      for (int i = 0; i < 16; ++i) f[i] = bf16x2_to_f32x2(p ? v[i].y : v[i].x);
+      // the first three butterfly stages on pairs, the signs s_i tracked at
+      // compile time; the last stage folds into the maximum, where signs do
+      // not matter: max(|a + b|, |a - b|) = |a| + |b| after rounding
+      fwht16_x2<3>(f, neg);
+#pragma unroll
+      for (int j = 0; j < 8; j += 2)
+        m = max3f(m, max3f(__fadd_rn(fabsf(f[j].x), fabsf(f[j + 8].x)), __fadd_rn(fabsf(f[j].y), fabsf(f[j + 8].y)),
+                           __fadd_rn(fabsf(f[j + 1].x), fabsf(f[j + 9].x))),
+                  __fadd_rn(fabsf(f[j + 1].y), fabsf(f[j + 9].y)));
     }
   }
   uint32_t mp = max(mplain & 0xFFFFu, mplain >> 16);
@@ -158,8 +163,9 @@ cudaError_t launch_amax(const void* x, int64_t R, int64_t C, int64_t ld, int rht
   if (rht) {
     const int64_t items = (R / 16) * (C / 4);
     const int64_t blocks = (items + 255) / 256;
-    // two waves of 3 CTAs per SM: measured 3% faster than one resident wave
-    const int grid = static_cast<int>(blocks < 6LL * num_sms ? blocks : 6LL * num_sms);
+    // two waves of 2 CTAs per SM (116 registers: the pair transform's 32 floats
+    // without spills); measured 4-6% faster than 3 CTAs per SM with spills
+    const int grid = static_cast<int>(blocks < 4LL * num_sms ? blocks : 4LL * num_sms);
     if (rht == 2)
       amax_rht_kernel<true><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), R, C, ld, out);
     else

@@ -236,6 +236,13 @@ __device__ __forceinline__ float2 bf16x2_to_f32x2(uint32_t w) {
   return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
+// max(a, b, c) in one instruction (a NaN operand is ignored, as fmaxf does).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // max(|a|, |b|, |c|) in one instruction.
 __device__ __forceinline__ float max3_abs(float a, float b, float c) {
   float d;
@@ -261,11 +268,13 @@ __device__ __forceinline__ float absmax16(const float2 (&v)[16]) {
 // (sa*(va - vb), sa*(va + vb)) otherwise; round-to-nearest is symmetric, so
 // the registers hold the true results up to those signs, bit for bit.  After
 // unrolling the signs are compile-time constants.
+// STAGES < 4 stops after the first STAGES stages (h = 1 .. 2^(STAGES-1)).
+template <int STAGES = 4>
 __device__ __forceinline__ void fwht16_x2(float2 (&v)[16], bool (&neg)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) neg[i] = rht_negates(i);
 #pragma unroll
-  for (int h = 1; h < 16; h <<= 1) {
+  for (int h = 1; h < (1 << STAGES); h <<= 1) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       if ((j & h) == 0) {
