@@ -1,5 +1,7 @@
 """Parity at the workloads' full sizes, in the launch configuration bench.py
-times (CTA-pair GEMM kernel, one-pass amax, the linear-layer C entry points).
+times (CTA-pair GEMM kernel, one-pass amax, the linear-layer C entry points,
+and the data-parallel layer with its one-read ROWCOL quantizer and second
+stream).
 
 Every quantized operand is compared with the oracle byte for byte over the
 whole tensor; GEMM outputs on 4096 seeded sampled entries (plus corners),
@@ -145,3 +147,18 @@ def test_fullsize_large_outlier_workload():
     _check_sampled(api.gemm(xr, wr, api.OUT_BF16), cx, sx, _gs(ax), cwr, swr, _gs(aw), True, "fprop", 31)
     _check_sampled(api.gemm(gr, wc, api.OUT_BF16), cg, sg, _gs(ag), cwc, swc, _gs(aw), True, "dgrad", 32)
     _check_sampled(api.gemm(gc, xc, api.OUT_F32), cgc, sgc, _gs(agr), cxc, sxc, _gs(axr), False, "wgrad", 33)
+    # the launch configuration bench.py times: the data-parallel layer on one rank, with X's
+    # one-read ROWCOL quantizer and the second stream (W's branch, the dY row copy beside wgrad)
+    from nvfp4_bit_microscaled_b200.dp import DataParallelLinear
+    layer = DataParallelLinear(T, Cin, Cout, "cuda")
+    Y = layer.forward(Xd, Wd)
+    dX, dW = layer.backward(Gd, seed)
+    torch.cuda.synchronize()
+    assert list(layer.amax_x.cpu().numpy()) == [ax, axr] and list(layer.amax_dy.cpu().numpy()) == [ag, agr]
+    for q, codes, sf, a, name in ((layer.x_row, cx, sx, ax, "layer X row"), (layer.x_col, cxc, sxc, axr, "layer X col"),
+                                  (layer.w_row, cwr, swr, aw, "layer W row"), (layer.w_col, cwc, swc, aw, "layer W col"),
+                                  (layer.dy_row, cg, sg, ag, "layer dY row"), (layer.dy_col, cgc, sgc, agr, "layer dY col")):
+        assert_q_equal(q, codes, sf, a, name)
+    _check_sampled(Y, cx, sx, _gs(ax), cwr, swr, _gs(aw), True, "layer Y", 34)
+    _check_sampled(dX, cg, sg, _gs(ag), cwc, swc, _gs(aw), True, "layer dX", 35)
+    _check_sampled(dW, cgc, sgc, _gs(agr), cxc, sxc, _gs(axr), False, "layer dW", 36)
