@@ -225,6 +225,10 @@ nvfp4_status nvfp4_mx_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D
  * GEMM, whose tensor-pipe work it overlaps.  Each call forks from and joins
  * back to `stream` with events of its own, so the calls stay stream-ordered
  * on `stream` (also under stream capture, as a fork/join in the graph).
+ * Calls from several host threads share the device's side stream: their
+ * branches run one after another there, each still ordered by its own
+ * events.  Capture these calls from one thread at a time (two captures
+ * cannot share the side stream).
  */
 size_t nvfp4_linear_workspace_bytes(int64_t T, int64_t Cin, int64_t Cout);
 nvfp4_status nvfp4_linear_fwd(const void* X, const void* W, int64_t T, int64_t Cin, int64_t Cout, void* Y,
