@@ -130,3 +130,35 @@ def test_dp_layer_back_to_back_steps_match_serial_steps():
         got.append((Y, dX, dW))
     torch.cuda.synchronize()
     _assert_same(got, ref)
+
+
+def test_two_host_threads_share_the_side_stream():
+    # each thread: its own workspace and caller stream; the library's side stream is shared
+    import threading
+    steps = _steps(4)
+    ref = _serial(steps)
+    got = [_outs() for _ in steps]
+    torch.cuda.synchronize()
+    errors = []
+
+    def worker(idx):
+        try:
+            ws = api.LinearWorkspace(T, CIN, COUT, "cuda")
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                for i in idx:
+                    X, W, dY = steps[i]
+                    _one_step(X, W, dY, ws, 77 + i, got[i])
+            s.synchronize()
+        except Exception as e:   # reported by the main thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(idx,)) for idx in ((0, 2), (1, 3))]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not any(t.is_alive() for t in threads), "a worker thread did not finish"
+    assert not errors, errors
+    torch.cuda.synchronize()
+    _assert_same(got, ref)
