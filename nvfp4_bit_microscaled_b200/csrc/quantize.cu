@@ -387,8 +387,9 @@ __global__ void __launch_bounds__(256, 2) quant_col_rn_kernel(const uint16_t* __
 // wgrad, and two kernels would read it twice.  Warp item: 64 tokens x 128
 // channels, in four bands of 16 rows.  For each band, lane l loads its 4
 // channels of the 16 rows (8-byte loads, 256 coalesced bytes per row per warp)
-// and quantizes their column blocks from registers, as the column kernel does
-// (RHT optional, scaled by the column copy's amax); it also stages the band in
+// and quantizes their column blocks from registers, two channels at a time as
+// FP32 pairs (RHT optional, signs tracked at compile time, as the SR column
+// kernel does; scaled by the column copy's amax); it also stages the band in
 // shared memory, from which lanes read the band's 16 x 8 row blocks of 16
 // channels (two 16-byte reads each) and quantize them as the row kernel does
 // (scaled by the row copy's amax).  A non-finite amax flags its copy (R25).
@@ -448,28 +449,42 @@ __global__ void __launch_bounds__(256, 2) quant_rowcol_kernel(
       for (int i = 0; i < 16; ++i) *reinterpret_cast<uint2*>(&bw[i][8 * lane]) = raw[i];
       if (!flag_col && lane_ok) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {   // column blocks: channel c0 + c, tokens tbase .. + 15
-          float v[16];
+        for (int p = 0; p < 2; ++p) {   // column blocks of channels c0 + 2p, c0 + 2p + 1 as FP32 pairs
+          float2 v[16];
+          bool neg[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const uint32_t w = (c < 2) ? raw[i].x : raw[i].y;
-            v[i] = __uint_as_float((c & 1) ? (w & 0xFFFF0000u) : (w << 16));
-            if (RHT && rht_negates(i)) v[i] = -v[i];  // s_i x_i
+            v[i] = bf16x2_to_f32x2(p ? raw[i].y : raw[i].x);
+            neg[i] = false;
           }
-          float m = 0.0f;
+          float m0, m1;
           if (RHT) {
-            m = __fmul_rn(fwht16_absmax<true>(v), 0.25f);
+            fwht16_x2(v, neg);
+            m0 = __fmul_rn(absmax16<false>(v), 0.25f);
+            m1 = __fmul_rn(absmax16<true>(v), 0.25f);
+            const float2 q4 = make_float2(0.25f, 0.25f);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.25f);
+            for (int i = 0; i < 16; ++i) v[i] = __fmul2_rn(v[i], q4);
           } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+            m0 = absmax16<false>(v);
+            m1 = absmax16<true>(v);
           }
-          const BlockScale bs = block_scale_t(m, se_col, r_col);
-          sfw[c] |= bs.sf << (8 * tb);
+          const BlockScale b0 = block_scale_t(m0, se_col, r_col), b1 = block_scale_t(m1, se_col, r_col);
+          sfw[2 * p] |= b0.sf << (8 * tb);
+          sfw[2 * p + 1] |= b1.sf << (8 * tb);
+          const float2 rp = make_float2(b0.r, b1.r), rn = make_float2(-b0.r, -b1.r);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], bs.r);
-          reinterpret_cast<uint2*>(col_data + (c0 + c) * half_r + t0 / 2)[tb] = make_uint2(pack8(v), pack8(v + 8));
+          for (int i = 0; i < 16; ++i) v[i] = __fmul2_rn(v[i], neg[i] ? rn : rp);
+          const uint32_t a0 = clear_negative_zero(
+              f32x8_to_e2m1x8(v[0].x, v[1].x, v[2].x, v[3].x, v[4].x, v[5].x, v[6].x, v[7].x));
+          const uint32_t a1 = clear_negative_zero(
+              f32x8_to_e2m1x8(v[8].x, v[9].x, v[10].x, v[11].x, v[12].x, v[13].x, v[14].x, v[15].x));
+          const uint32_t e0 = clear_negative_zero(
+              f32x8_to_e2m1x8(v[0].y, v[1].y, v[2].y, v[3].y, v[4].y, v[5].y, v[6].y, v[7].y));
+          const uint32_t e1 = clear_negative_zero(
+              f32x8_to_e2m1x8(v[8].y, v[9].y, v[10].y, v[11].y, v[12].y, v[13].y, v[14].y, v[15].y));
+          reinterpret_cast<uint2*>(col_data + (c0 + 2 * p) * half_r + t0 / 2)[tb] = make_uint2(a0, a1);
+          reinterpret_cast<uint2*>(col_data + (c0 + 2 * p + 1) * half_r + t0 / 2)[tb] = make_uint2(e0, e1);
         }
       }
       __syncwarp();
