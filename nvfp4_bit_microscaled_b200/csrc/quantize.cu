@@ -42,6 +42,30 @@ __device__ __noinline__ void flag_copy(uint8_t* __restrict__ data, int64_t rows,
   }
 }
 
+// Sixteen BF16 values (a, then b) as eight FP32 pairs, element 2k in y[k].x.
+__device__ __forceinline__ void unpack16_x2(uint4 a, uint4 b, float2 (&y)[8]) {
+  y[0] = bf16x2_to_f32x2(a.x); y[1] = bf16x2_to_f32x2(a.y); y[2] = bf16x2_to_f32x2(a.z); y[3] = bf16x2_to_f32x2(a.w);
+  y[4] = bf16x2_to_f32x2(b.x); y[5] = bf16x2_to_f32x2(b.y); y[6] = bf16x2_to_f32x2(b.z); y[7] = bf16x2_to_f32x2(b.w);
+}
+
+// max |y| over the sixteen values of unpack16_x2 (finite inputs).
+__device__ __forceinline__ float absmax16_x2(const float2 (&y)[8]) {
+  float m = max3_abs(y[0].x, y[0].y, y[1].x);
+#pragma unroll
+  for (int k = 1; k < 7; ++k) m = max3_abs(m, y[k].y, y[k + 1].x);
+  return max3_abs(m, y[7].y, 0.0f);
+}
+
+// The sixteen values times r, round-to-nearest E2M1 codes, two words.
+__device__ __forceinline__ uint2 scale_pack16_x2(float2 (&y)[8], float r) {
+  const float2 r2 = make_float2(r, r);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) y[k] = __fmul2_rn(y[k], r2);
+  return make_uint2(
+      clear_negative_zero(f32x8_to_e2m1x8(y[0].x, y[0].y, y[1].x, y[1].y, y[2].x, y[2].y, y[3].x, y[3].y)),
+      clear_negative_zero(f32x8_to_e2m1x8(y[4].x, y[4].y, y[5].x, y[5].y, y[6].x, y[6].y, y[7].x, y[7].y)));
+}
+
 __device__ __forceinline__ void unpack8(uint4 v, float* f) {
   f[0] = bf16_bits_to_f32(v.x & 0xFFFFu); f[1] = bf16_bits_to_f32(v.x >> 16);
   f[2] = bf16_bits_to_f32(v.y & 0xFFFFu); f[3] = bf16_bits_to_f32(v.y >> 16);
@@ -141,16 +165,13 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
         w0 = clear_negative_zero(f32x8_to_e2m1x8(y[0].x, y[0].y, y[1].x, y[1].y, y[2].x, y[2].y, y[3].x, y[3].y));
         w1 = clear_negative_zero(f32x8_to_e2m1x8(y[4].x, y[4].y, y[5].x, y[5].y, y[6].x, y[6].y, y[7].x, y[7].y));
       } else {
-        const uint32_t mb = max(absmax_bits8(v[u][0]), absmax_bits8(v[u][1]));
-        const BlockScale bs0 = block_scale_t(bf16_bits_to_f32(mb), s_enc, r_tbl);
+        float2 y[8];
+        unpack16_x2(v[u][0], v[u][1], y);
+        const BlockScale bs0 = block_scale_t(absmax16_x2(y), s_enc, r_tbl);
         sfb = bs0.sf;
-        float y[16];
-        unpack8(v[u][0], y);
-        unpack8(v[u][1], y + 8);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(y[i], bs0.r);
-        w0 = pack8(y);
-        w1 = pack8(y + 8);
+        const uint2 w = scale_pack16_x2(y, bs0.r);
+        w0 = w.x;
+        w1 = w.y;
       }
       if (ok[u]) *reinterpret_cast<uint2*>(data + rr[u] * half_c + bb[u] * 8) = make_uint2(w0, w1);
       uint32_t word = ok[u] ? (sfb << (8 * (lane & 3))) : 0u;
@@ -499,15 +520,11 @@ __global__ void __launch_bounds__(256, 2) quant_rowcol_kernel(
             v0 = *reinterpret_cast<const uint4*>(&bw[i][32 * b]);
             v1 = *reinterpret_cast<const uint4*>(&bw[i][32 * b + 16]);
           }
-          const uint32_t mb = max(absmax_bits8(v0), absmax_bits8(v1));
-          const BlockScale bs = block_scale_t(bf16_bits_to_f32(mb), se_row, r_row);
-          float y[16];
-          unpack8(v0, y);
-          unpack8(v1, y + 8);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) y[e] = __fmul_rn(y[e], bs.r);
-          const uint32_t w0 = pack8(y), w1 = pack8(y + 8);
-          if (ok) *reinterpret_cast<uint2*>(row_data + (tbase + i) * half_c + cb / 2) = make_uint2(w0, w1);
+          float2 y[8];
+          unpack16_x2(v0, v1, y);
+          const BlockScale bs = block_scale_t(absmax16_x2(y), se_row, r_row);
+          const uint2 w = scale_pack16_x2(y, bs.r);
+          if (ok) *reinterpret_cast<uint2*>(row_data + (tbase + i) * half_c + cb / 2) = w;
           // lanes 4k .. 4k+3 hold four consecutive blocks of the row: one scale word
           uint32_t word = ok ? (bs.sf << (8 * (b & 3))) : 0u;
           word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
