@@ -121,6 +121,50 @@ def test_quantize_row_sr_distribution_matches_worked_example():
     assert abs(up - 0.40625) < 5 * 0.5 / np.sqrt(sel.sum())
 
 
+def _grid_blocks(rows, blocks_per_row):
+    # every 16-element block: max 6 * 2^k (so its E4M3 scale is exactly 2^k with S_enc = 1) and
+    # values on the E2M1 grid, on its binade boundaries and at its midpoints, with random signs;
+    # one element of 2688 fixes the tensor amax (S_enc = 2688 / 2688 = 1)
+    vals = np.array([6.0, 4.0, 3.0, 2.0, 1.5, 1.0, 0.5, 0.0, 5.0, 3.5, 2.5, 1.75, 1.25, 0.75, 0.25, 0.125],
+                    dtype=np.float32)
+    rng = np.random.default_rng(11)
+    x = np.empty((rows, 16 * blocks_per_row), dtype=np.float32)
+    for r in range(rows):
+        for b in range(blocks_per_row):
+            k = rng.integers(-6, 7)
+            blk = rng.permutation(vals) * np.float32(2.0 ** k)
+            blk[np.argmax(np.abs(blk))] = np.float32(6.0 * 2.0 ** k)
+            x[r, 16 * b:16 * b + 16] = blk * rng.choice(np.array([-1.0, 1.0], dtype=np.float32), 16)
+    x[0, 0] = 2688.0
+    return torch.from_numpy(x).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("seed", [1, 12345])
+def test_sr_on_grid_points_boundaries_and_midpoints(seed):
+    # the SR decision's directed roundings (fma.rp / add.rp on FP32 pairs) at the values where
+    # they matter: scaled values exactly on the grid (must not move), on the binade boundaries
+    # 1, 2, 4, 6 and at midpoints; row and column copies, bit-exact against the oracle
+    xb = _grid_blocks(64, 20)
+    a = O.amax(xb)
+    assert a == 2688.0
+    row, _ = api.quantize(dev(xb), api.ROW, api.amax(dev(xb)), sr=True, seed=seed)
+    assert_q_equal(row, *O.quantize_row(xb, a, sr=True, seed=seed), a, "row SR on grid values")
+    xt = xb.t().contiguous()      # the same blocks down the columns
+    at = O.amax(xt)
+    _, col = api.quantize(dev(xt), api.COL, api.amax(dev(xt)), sr=True, seed=seed)
+    assert_q_equal(col, *O.quantize_col(xt, at, sr=True, seed=seed), at, "column SR on grid values")
+    # values already on the grid come back unchanged, whatever the random words
+    data = row.data.cpu().numpy()
+    codes = np.empty((data.shape[0], data.shape[1] * 2), dtype=np.uint8)
+    codes[:, 0::2], codes[:, 1::2] = data & 15, data >> 4
+    cr, _ = O.quantize_row(xb, a)          # round to nearest: exact on grid values
+    on_grid = np.isin(np.abs(xb.float().numpy()) / np.repeat(
+        np.maximum(np.abs(xb.float().numpy()).reshape(64, -1, 16).max(axis=2), 1e-30) / 6.0, 16, axis=1),
+        [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    on_grid[0, :16] = False                # block 0 holds the tensor max
+    assert np.array_equal(codes[on_grid], np.asarray(cr)[on_grid])
+
+
 # ------------------------------------------------------------------ column-wise
 @pytest.mark.parametrize("name,x", _inputs())
 @pytest.mark.parametrize("rht,sr", [(False, False), (True, False), (False, True), (True, True)])
