@@ -215,9 +215,9 @@ nvfp4_status nvfp4_mx_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D
  * nvfp4_linear_fwd: amax and RHT amax of X (one pass) -> X row copy (RN) and X
  *   column copy with RHT (RN, kept for wgrad) from one read of X; amax(W) ->
  *   W 2D (row + column copies, RN); Y = gemm(Xq, Wq) in BF16.
- * nvfp4_linear_bwd: amax(dY) -> dY row copy with SR (seed); dX = gemm(dYq, W^T
- *   column copy) in BF16; amax_rht(dY) -> dY column copy with RHT and SR
- *   (seed); dW = gemm(dY^T q, X^T q) in FP32.
+ * nvfp4_linear_bwd: amax and RHT amax of dY (one pass) -> dY column copy with
+ *   RHT and SR (seed); dW = gemm(dY^T q, X^T q) in FP32, and beside it the dY
+ *   row copy with SR (seed); then dX = gemm(dYq, W^T column copy) in BF16.
  * Needs T, Cin, Cout multiples of 64.
  * Both calls run independent branches on a second stream that the library
  * creates once per device (non-blocking): in the forward, W's amax and 2D
@@ -256,7 +256,9 @@ nvfp4_status nvfp4_linear_bwd(const void* dY, int64_t T, int64_t Cin, int64_t Co
  *   - Returns NVFP4_ERR_WORKSPACE, before enqueuing anything, when the part
  *     of the linear workspace the forward uses (the scalars, the X row copy
  *     and both W copies) exceeds the scratch size.
- *   - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
+ *   - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call),
+ *     and creates no stream or event: every kernel runs on `stream`, one
+ *     after another.
  *   - The first call in each CUDA context looks up the scratch address in
  *     that context (cudaGetSymbolAddress, cached by the context's id); make
  *     that first call before any stream capture in the context.
