@@ -228,7 +228,9 @@ nvfp4_status nvfp4_mx_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* D
  * Calls from several host threads share the device's side stream: their
  * branches run one after another there, each still ordered by its own
  * events.  Capture these calls from one thread at a time (two captures
- * cannot share the side stream).
+ * cannot share the side stream), and make the first call on a device and
+ * host thread outside any capture: it creates the side stream and that
+ * thread's two events.
  */
 size_t nvfp4_linear_workspace_bytes(int64_t T, int64_t Cin, int64_t Cout);
 nvfp4_status nvfp4_linear_fwd(const void* X, const void* W, int64_t T, int64_t Cin, int64_t Cout, void* Y,
