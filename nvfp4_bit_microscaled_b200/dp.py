@@ -137,16 +137,13 @@ class DataParallelLinear:
             start = torch.cuda.Event()
             start.record(torch.cuda.current_stream())
         dW = d("gemm_wgrad", lambda: api.gemm(self.dy_col, self.x_col, api.OUT_F32, out=dW))
-        pending = None
-        if self.world > 1:
-            if dist.get_backend(self.group) == "nccl":
-                pending = dist.all_reduce(dW, op=dist.ReduceOp.SUM, group=self.group, async_op=True)
-            else:
-                d("allreduce_dw", lambda: self._all_reduce(dW, dist.ReduceOp.SUM))
         # the dY row copy (SR) on the side stream, next to the wgrad GEMM: the
-        # quantizer is bound by the integer ALU pipe, the GEMM by the tensor pipe
+        # quantizer is bound by the integer ALU pipe, the GEMM by the tensor pipe.
+        # Enqueued before the dW all-reduce, so that a host-staged (gloo) reduce
+        # does not hold it back.
         row_sr = lambda: d("quant_row_sr", lambda: api.quantize(dY, api.ROW, self.amax_dy[0:1], sr=True, seed=seed,
                                                                 row_out=self.dy_row, row0=self.row0))
+        done = None
         if side is None:
             row_sr()
         else:
@@ -155,6 +152,13 @@ class DataParallelLinear:
                 row_sr()
                 done = torch.cuda.Event()
                 done.record(side)
+        pending = None
+        if self.world > 1:
+            if dist.get_backend(self.group) == "nccl":
+                pending = dist.all_reduce(dW, op=dist.ReduceOp.SUM, group=self.group, async_op=True)
+            else:
+                d("allreduce_dw", lambda: self._all_reduce(dW, dist.ReduceOp.SUM))
+        if done is not None:
             torch.cuda.current_stream().wait_event(done)
         dX = d("gemm_dgrad", lambda: api.gemm(self.dy_row, self.w_col, api.OUT_BF16, out=dX))
         if pending is not None:
