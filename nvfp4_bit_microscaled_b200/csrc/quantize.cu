@@ -779,7 +779,9 @@ cudaError_t launch_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, co
                              cudaStream_t s) {
   const int64_t S = C / 16, sp = (S + 3) / 4 * 4;
   const int64_t warp_items = R * ((S + 31) / 32);
-  const int grid = grid_for(warp_items, 8 * 2, num_sms, 8);
+  // up to 32 CTAs per SM over the launch (short-lived CTAs, 4 resident at a
+  // time): measured 2.5-2.8% faster than 8 for the SR and RN row copies
+  const int grid = grid_for(warp_items, 8 * 2, num_sms, 32);
   const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
   auto* xs = static_cast<const uint16_t*>(x);
   auto* d = static_cast<uint8_t*>(data);
@@ -829,7 +831,9 @@ cudaError_t launch_quant_rowcol(const void* x, int64_t R, int64_t C, int64_t ld,
                                 void* col_data, void* col_scales, float* col_gs, int num_sms, cudaStream_t s) {
   const int64_t S = R / 16;
   const int64_t warp_items = ((S + 3) / 4) * ((C + 127) / 128);
-  const int grid = grid_for(warp_items, 8, num_sms, 8);
+  // up to 16 CTAs per SM over the launch (2 resident at a time): measured 3%
+  // faster than 8 at 32768 x 8192
+  const int grid = grid_for(warp_items, 8, num_sms, 16);
   auto* xs = static_cast<const uint16_t*>(x);
   auto* rd = static_cast<uint8_t*>(row_data);
   auto* rf = static_cast<uint8_t*>(row_scales);
