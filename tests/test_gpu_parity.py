@@ -181,6 +181,59 @@ def test_quantize_col(name, x, rht, sr):
     assert_q_equal(col, codes, sf, a, f"{name} col rht={rht} sr={sr}")
 
 
+@pytest.mark.parametrize("R,C", [(48, 100), (32, 4), (48, 1028), (80, 1540)])
+@pytest.mark.parametrize("rht,sr", [(False, False), (True, False), (False, True), (True, True)])
+def test_quantize_col_four_channel_tail(R, C, rht, sr):
+    # C % 8 == 4: a strip's last four channels are not a whole 16-byte copy and
+    # are read from global memory; with C = 4, 1028 and 1540 the last
+    # 512-channel strip has nothing to copy at all.  The amax is the oracle's,
+    # passed in (the device RHT amax wants C % 8 == 0).
+    # rows padded to C + 4 channels: the row stride must be a multiple of 8
+    x = synth.gradients(R, C, 51)
+    a = O.amax_rht(x) if rht else O.amax(x)
+    amax_dev = torch.tensor([a], dtype=torch.float32, device="cuda")
+    xp = torch.zeros(R, C + 4, dtype=torch.bfloat16, device="cuda")
+    xp[:, :C] = dev(x)
+    _, col = api.quantize(xp[:, :C], api.COL, amax_dev, rht=rht, sr=sr, seed=78)
+    codes, sf = O.quantize_col(x, a, rht=rht, sr=sr, seed=78)
+    assert_q_equal(col, codes, sf, a, f"col tail {R}x{C} rht={rht} sr={sr}")
+
+
+@pytest.mark.parametrize("rht,sr", [(False, False), (True, False), (False, True), (True, True)])
+def test_quantize_col_strided_rows(rht, sr):
+    # a row stride past C: the staged copies read each row from its own stride
+    big = synth.gradients(96, 776, 53)
+    x = dev(big)[:, :768]
+    xc = big[:, :768].contiguous()
+    a = O.amax_rht(xc) if rht else O.amax(xc)
+    _, col = api.quantize(x, api.COL, api.amax(x, rht=rht), rht=rht, sr=sr, seed=79)
+    codes, sf = O.quantize_col(xc, a, rht=rht, sr=sr, seed=79)
+    assert_q_equal(col, codes, sf, a, f"col strided rht={rht} sr={sr}")
+
+
+@pytest.mark.parametrize("rht,sr", [(True, True), (True, False), (False, True)])
+def test_quantize_col_many_items_per_cta(rht, sr):
+    # 8192 tokens x 1600 channels: 2048 items of 16 tokens x a 512-channel
+    # strip (the last strip 64 channels), more than three per resident CTA, so
+    # every stage buffer is refilled and its barrier runs through both phases
+    x = synth.gradients(8192, 1600, 54)
+    a = O.amax_rht(x) if rht else O.amax(x)
+    _, col = api.quantize(dev(x), api.COL, api.amax(dev(x), rht=rht), rht=rht, sr=sr, seed=80)
+    codes, sf = O.quantize_col(x, a, rht=rht, sr=sr, seed=80)
+    assert_q_equal(col, codes, sf, a, f"col 8192x1600 rht={rht} sr={sr}")
+
+
+@pytest.mark.parametrize("rht", [False, True])
+def test_quantize_rowcol_many_items_per_cta(rht):
+    x = synth.activations(8192, 1600, 55)
+    a, ar = O.amax(x), O.amax_rht(x)
+    amax_dev = api.amax(dev(x), rht=2) if rht else api.amax(dev(x))
+    row, col = api.quantize(dev(x), api.ROWCOL, amax_dev, rht=rht)
+    assert_q_equal(row, *O.quantize_row(x, a), a, "rowcol 8192x1600 row")
+    ac = ar if rht else a
+    assert_q_equal(col, *O.quantize_col(x, ac, rht=rht), ac, f"rowcol 8192x1600 col rht={rht}")
+
+
 def test_quantize_rowcol():
     x = synth.gradients(192, 256, 41)
     a = O.amax(x)
