@@ -251,10 +251,17 @@ class AloneTimer:
     """timer(kind, fn) that times each library call alone, after the step's
     timed region: the device is idle before every launch (so no kernel of the
     other stream runs beside it), L2 is flushed with a 256 MB write, and the
-    call is launched `reps` times; collectives run once, untimed."""
+    call is launched `reps` times; collectives run once, untimed.
 
-    def __init__(self, device, reps=5):
+    The device would reach the start event as soon as the flush ends, while
+    the host may still be inside the call (argument marshalling, the launch):
+    that gap would be timed as the kernel's.  A device-side wait of `hold_cycles`
+    after the flush keeps the device busy until the call is enqueued, as it is
+    in the back-to-back step."""
+
+    def __init__(self, device, reps=5, hold_cycles=1_000_000):
         self.reps = reps
+        self.hold_cycles = hold_cycles
         self.ms = {}
         self.scratch = torch.empty(256 << 20, dtype=torch.uint8, device=device)
 
@@ -266,6 +273,8 @@ class AloneTimer:
         for _ in range(self.reps):
             torch.cuda.synchronize()
             self.scratch.fill_(1)
+            if self.hold_cycles:
+                torch.cuda._sleep(self.hold_cycles)
             s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s.record()
             out = fn()
@@ -423,8 +432,9 @@ def time_step(wl, args, rank, world, device, clocks=True):
                     "stream, so overlapping shares can sum above 1"),
         "kernels_alone": kernels_alone,
         "kernels_alone_note": ("each call once more after the timed region, alone on an idle device, L2 "
-                               "flushed before each of 5 launches: the kernel's own rate, without the "
-                               "second stream's overlap"),
+                               "flushed before each of 5 launches, each enqueued behind a short device-side "
+                               "wait so that the host's launch time is not timed: the kernel's own rate, "
+                               "without the second stream's overlap"),
         "_fprop": (gf["gemm_fprop"], avg_ms["gemm_fprop"], fpeak, fpeak_src),
         "_clocks": clk.summary(),
         "_tensors": (X, W, dY),
