@@ -48,7 +48,9 @@ def lib():
             "orc_e4m3_encode_rn_sat": (ctypes.c_int, [ctypes.c_float]),
             "orc_e2m1_encode_sr": (ctypes.c_int, [ctypes.c_float, ctypes.c_uint32]),
             "orc_philox4x32_10": (None, [_u32p, _u32p, _u32p]),
-            "orc_sr_word": (ctypes.c_uint32, [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_uint32]),
+            "orc_sr_block_words": (None, [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_uint32, _u32p]),
+            "orc_sr_draw16": (ctypes.c_uint32, [ctypes.c_uint32, ctypes.c_int]),
+            "orc_sr_block_draws": (None, [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_uint32, _u32p]),
             "orc_rht_signs": (None, [_f32p]),
             "orc_rht16_f32": (None, [_f32p, _f32p]),
             "orc_rht16_f64": (None, [_f64p, _f64p]),
@@ -111,8 +113,9 @@ def e4m3_encode_rn_sat(d):
     return lib().orc_e4m3_encode_rn_sat(float(d))
 
 
-def e2m1_encode_sr(y, w):
-    return lib().orc_e2m1_encode_sr(float(y), int(w) & 0xFFFFFFFF)
+def e2m1_encode_sr(y, r16):
+    """Stochastic rounding of y with the 16-bit draw r16 (R10)."""
+    return lib().orc_e2m1_encode_sr(float(y), int(r16) & 0xFFFF)
 
 
 # ---------------------------------------------------------------- philox / rht
@@ -124,8 +127,23 @@ def philox4x32_10(ctr, key):
     return out
 
 
-def sr_word(seed, idx, domain):
-    return lib().orc_sr_word(int(seed), int(idx), int(domain))
+def sr_block_words(seed, g, domain):
+    """The four Philox words of the block keyed g (R11)."""
+    out = np.zeros(4, dtype=np.uint32)
+    lib().orc_sr_block_words(int(seed), int(g), int(domain), _p(out, _u32p))
+    return out
+
+
+def sr_draw16(word, q):
+    """The 16-bit draw of element q (0..3) of a word (R10)."""
+    return lib().orc_sr_draw16(int(word) & 0xFFFFFFFF, int(q))
+
+
+def sr_block_draws(seed, g, domain):
+    """The 16-bit draws of the sixteen elements of the block keyed g."""
+    out = np.zeros(16, dtype=np.uint32)
+    lib().orc_sr_block_draws(int(seed), int(g), int(domain), _p(out, _u32p))
+    return out
 
 
 def rht_signs():

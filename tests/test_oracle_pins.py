@@ -101,23 +101,75 @@ def test_philox_known_answers():
         assert list(out) == v[6:10]
 
 
-def test_sr_word_keying():
+def test_sr_block_keying():
+    # R11: one generator call per 16-element block, the counter's low and high
+    # words from g, its third word the domain
     seed = 0x0123456789ABCDEF
-    for idx in (0, 1, 2, 3, 4, 7, 2 ** 33 + 5):
-        g = idx >> 2
+    for g in (0, 1, 2, 5, 2 ** 33 + 5):
         out = O.philox4x32_10([g & 0xFFFFFFFF, g >> 32, 1, 0], [seed & 0xFFFFFFFF, seed >> 32])
-        assert O.sr_word(seed, idx, 1) == out[idx & 3]
+        assert list(O.sr_block_words(seed, g, 1)) == list(out)
+        draws = O.sr_block_draws(seed, g, 1)
+        assert [int(d) for d in draws] == [O.sr_draw16(out[i // 4], i % 4) for i in range(16)]
 
 
-# ----------------------------------------------------------------- stochastic rounding
+def _rev(x, n):
+    return int(format(x, f"0{n}b")[::-1], 2)
+
+
+def test_sr_draw_is_a_bijection_of_its_sixteen_bits():
+    # R10: each element's draw is a bijection of the 16 bits it reads, so a
+    # uniform word gives a uniform draw; the two elements that read the same 16
+    # bits get them in opposite orders, and the other two bytes never enter
+    for q in range(4):
+        lo_byte, hi_byte = (0, 2) if q < 2 else (1, 3)
+        other = [k for k in range(4) if k not in (lo_byte, hi_byte)]
+        seen = np.zeros(1 << 16, dtype=np.int32)
+        for lo in range(256):
+            for hi in range(256):
+                noise = ((lo * 7 + hi) & 0xFF) << (8 * other[0]) | ((hi * 13 + 5) & 0xFF) << (8 * other[1])
+                d = O.sr_draw16((lo << (8 * lo_byte)) | (hi << (8 * hi_byte)) | noise, q)
+                natural = (hi << 8) | lo
+                assert d == (natural if q % 2 == 0 else _rev(natural, 16)), (q, lo, hi)
+                seen[d] += 1
+        assert np.all(seen == 1), q
+
+
+def test_sr_probability_is_floor_of_p_times_2_16():
+    # R10, pinned by counting: over the 2^16 draws, y rounds up exactly
+    # floor(p * 2^16) times, p = (|y| - lo) / step computed exactly in rationals
+    from fractions import Fraction
+    rng = np.random.default_rng(3)
+    ys = [0.0, 0.25, 0.3, 0.5, 0.74, 1.1, 1.999, 2.0, 2.5, 3.4, 3.999, 4.0, 5.0, 5.999, 6.0, 6.3, -0.3, -2.5]
+    ys += [float(v) for v in rng.uniform(0, 6, 40).astype(np.float32)]
+    grid = [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+    for y in ys:
+        y = float(np.float32(y))
+        a = Fraction(abs(y))
+        if a >= 6:
+            want_up, lo = 0, Fraction(6)
+        else:
+            step = Fraction(1, 2) if a < 2 else (Fraction(1) if a < 4 else Fraction(2))
+            lo = (a // step) * step
+            want_up = int(((a - lo) / step) * 65536)        # floor
+        codes = [O.e2m1_encode_sr(y, r) for r in range(1 << 16)]
+        mags = [O.e2m1_decode(c & 7) for c in codes]
+        ups = sum(1 for m in mags if m > lo)
+        assert ups == want_up, (y, ups, want_up)
+        assert all(m in (float(lo), float(min(lo + (step if a < 6 else 0), 6))) for m in mags) if a < 6 else \
+            all(m == 6.0 for m in mags)
+        # the draws that round up are the largest ones
+        if 0 < ups < 65536:
+            assert mags[65535 - ups] == float(lo) and mags[65536 - ups] > float(lo)
+
+
 def test_sr_worked_example():
-    # 3.4 between 3 and 4: P(4) = 0.4, P(3) = 0.6 (the page's worked example)
+    # 3.4 between 3 and 4: P(4) = 0.4, P(3) = 0.6 (the page's worked example),
+    # to within the draws' resolution of 2^-16
     (val, lo, hi, p_lo, p_hi), = [[float(t) for t in r] for r in _rows("sr_worked_example.txt")]
     n = 1 << 16
     ups = 0
-    for i in range(n):
-        c = O.e2m1_encode_sr(val, (i << 16) | 0xFF)   # u = i / 2^16, evenly spaced
-        v = O.e2m1_decode(c)
+    for r in range(n):
+        v = O.e2m1_decode(O.e2m1_encode_sr(val, r))
         assert v in (lo, hi)
         ups += v == hi
     assert abs(ups / n - p_hi) < 2.0 / n
@@ -368,24 +420,28 @@ def test_row_block_quantize_equals_slice_of_whole_tensor(row0, rows):
 
 
 def test_row_offset_reaches_the_counter_high_word():
-    # a block whose element indices / 4 pass 2^32: its words are those of the
-    # whole-tensor indices, read one by one from the generator
+    # blocks whose counters g = (row0 + r) * C/16 + b pass 2^32: their draws are
+    # those of the whole tensor's blocks, read one by one from the generator
     C, rows = 64, 16
-    row0 = (1 << 34) // C - 8            # the block straddles element index 2^34
+    row0 = (1 << 36) // C - 8            # the rows straddle block counter 2^32
     x = synth.gradients(rows, C, 32)
     a = O.amax(x)
     codes, sf = O.quantize_row(x, a, sr=True, seed=5, row0=row0)
     S_enc = float(O.global_scales(a)[0])
     xf = x.float().numpy()
+    crossed = False
     for r in (0, 7, 8, 15):
         for b in range(C // 16):
+            g = (row0 + r) * (C // 16) + b
+            crossed |= g >= 1 << 32
+            draws = O.sr_block_draws(5, g, 0)
             blk = xf[r, b * 16:(b + 1) * 16]
             sb = O.e4m3_decode(sf[r, b])
             for i in range(16):
-                idx = (row0 + r) * C + b * 16 + i
                 y = np.float32(blk[i]) * (np.float32(S_enc) / np.float32(sb)) if sb else np.float32(0)
-                want = O.e2m1_encode_sr(float(y), O.sr_word(5, idx, 0)) if sb else 0
+                want = O.e2m1_encode_sr(float(y), int(draws[i])) if sb else 0
                 assert codes[r, b * 16 + i] == want, (r, b, i)
+    assert crossed
 
 
 # ----------------------------------------------------------------- non-finite inputs (R25)
