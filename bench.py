@@ -251,7 +251,8 @@ class AloneTimer:
     """timer(kind, fn) that times each library call alone, after the step's
     timed region: the device is idle before every launch (so no kernel of the
     other stream runs beside it), L2 is flushed with a 256 MB write, and the
-    call is launched `reps` times; collectives run once, untimed.
+    call is launched once untimed, then `reps` times timed; collectives run
+    once, untimed.
 
     The device would reach the start event as soon as the flush ends, while
     the host may still be inside the call (argument marshalling, the launch):
@@ -268,8 +269,8 @@ class AloneTimer:
     def __call__(self, kind, fn):
         if kind.startswith("allreduce"):
             return fn()
+        out = fn()   # untimed: the call's first-use work (an output allocation, a descriptor) is done here
         times = []
-        out = None
         for _ in range(self.reps):
             torch.cuda.synchronize()
             self.scratch.fill_(1)

@@ -60,6 +60,7 @@ PROTOTYPES = {
     "nvfp4_mx_quantize": (_int, [_vp, _i64, _i64, _i64, _tp, _vp]),
     "nvfp4_mx_gemm": (_int, [_tp, _tp, _vp, _int, _i64, _vp]),
     "nvfp4_selftest_scale_division": (_int, [_c.POINTER(_c.c_uint64), _c.POINTER(_c.c_uint64)]),
+    "nvfp4_selftest_sr_rounding": (_int, [_c.POINTER(_c.c_uint64), _c.POINTER(_c.c_uint64)]),
 }
 
 _LIB = None

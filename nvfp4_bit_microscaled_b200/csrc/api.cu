@@ -282,6 +282,18 @@ nvfp4_status nvfp4_selftest_scale_division(uint64_t* bad_quotients, uint64_t* ba
   return st;
 }
 
+nvfp4_status nvfp4_selftest_sr_rounding(uint64_t* mismatches, uint64_t* checked) {
+  if (!mismatches || !checked) return NVFP4_ERR_INVALID_ARG;
+  DeviceInfo di;
+  nvfp4_status st = device_info(&di);
+  if (st != NVFP4_OK) return st;
+  unsigned long long m = 0, c = 0;
+  st = cuda_status(nvfp4::selftest_sr(&m, &c));
+  *mismatches = m;
+  *checked = c;
+  return st;
+}
+
 int nvfp4_version(void) { return 1; }
 
 int nvfp4_last_cuda_error(const char** name) {

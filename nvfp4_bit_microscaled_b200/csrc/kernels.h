@@ -43,6 +43,10 @@ cudaError_t launch_quant_2d(const void* w, int64_t N, int64_t K, int64_t ld, con
 // non-negative finite float (synchronous, default stream).
 cudaError_t selftest_div6(unsigned long long* bad_quotients, unsigned long long* bad_codes, int num_sms);
 
+// Self-test: the stochastic-rounding conversion against its rule, every
+// 16-bit draw of every lane for a spread of values (synchronous).
+cudaError_t selftest_sr(unsigned long long* mismatches, unsigned long long* checked);
+
 // Zero the padding of a scale matrix (rows >= R or scale columns >= S).
 cudaError_t launch_sf_pad_zero(void* scales, int64_t R, int64_t S, cudaStream_t s);
 

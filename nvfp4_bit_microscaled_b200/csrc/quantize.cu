@@ -80,7 +80,7 @@ __device__ __forceinline__ void unpack8(uint4 v, float* f) {
 // Warp item: one row segment of 32 blocks (512 elements); lane = block.
 // Scale bytes of lanes 4j..4j+3 form one 32-bit word of the 128x4 tile layout.
 // ---------------------------------------------------------------------------
-// NARROW (SR only): every element index / 4 fits in 32 bits.
+// NARROW (SR only): every block counter (element index / 16) fits in 32 bits.
 template <bool SR, bool NARROW>
 __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
                                                           int64_t ld, const float* __restrict__ amax_dev,
@@ -144,7 +144,8 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
       uint32_t sfb;
       uint32_t w0, w1;
       if (SR) {
-        // elements (2k, 2k+1) as FP32 pairs: the scaling and the SR decision run packed
+        // elements (2k, 2k+1) as FP32 pairs: the scaling runs packed, the
+        // rounding in the conversion, four elements per random word
         const uint4 a = v[u][0], b = v[u][1];
         float2 y[8] = {bf16x2_to_f32x2(a.x), bf16x2_to_f32x2(a.y), bf16x2_to_f32x2(a.z), bf16x2_to_f32x2(a.w),
                        bf16x2_to_f32x2(b.x), bf16x2_to_f32x2(b.y), bf16x2_to_f32x2(b.z), bf16x2_to_f32x2(b.w)};
@@ -155,15 +156,15 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
         const BlockScale bs0 = block_scale_t(m, s_enc, r_tbl);
         sfb = bs0.sf;
         const float2 r2 = make_float2(bs0.r, bs0.r);
-        const uint64_t g = static_cast<uint64_t>(rr[u] * C + bb[u] * 16 + idx0) >> 2;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const u32x4 w = sr_words<NARROW>(g + q, kDomainRowSR, k0, k1);
-          y[2 * q] = sr_magnitude2<false>(__fmul2_rn(y[2 * q], r2), w.x, w.y);
-          y[2 * q + 1] = sr_magnitude2<false>(__fmul2_rn(y[2 * q + 1], r2), w.z, w.w);
-        }
-        w0 = clear_negative_zero(f32x8_to_e2m1x8(y[0].x, y[0].y, y[1].x, y[1].y, y[2].x, y[2].y, y[3].x, y[3].y));
-        w1 = clear_negative_zero(f32x8_to_e2m1x8(y[4].x, y[4].y, y[5].x, y[5].y, y[6].x, y[6].y, y[7].x, y[7].y));
+        for (int k = 0; k < 8; ++k) y[k] = __fmul2_rn(y[k], r2);
+        // one generator call per block: (idx0 + r*C)/16 + b (C and idx0 are multiples of 16)
+        const uint64_t g = (static_cast<uint64_t>(rr[u] * C + idx0) >> 4) + static_cast<uint64_t>(bb[u]);
+        const u32x4 w = sr_words<NARROW>(g, kDomainRowSR, k0, k1);
+        w0 = clear_negative_zero(sr_e2m1x4(y[0].x, y[0].y, y[1].x, y[1].y, w.x) |
+                                 (sr_e2m1x4(y[2].x, y[2].y, y[3].x, y[3].y, w.y) << 16));
+        w1 = clear_negative_zero(sr_e2m1x4(y[4].x, y[4].y, y[5].x, y[5].y, w.z) |
+                                 (sr_e2m1x4(y[6].x, y[6].y, y[7].x, y[7].y, w.w) << 16));
       } else {
         float2 y[8];
         unpack16_x2(v[u][0], v[u][1], y);
@@ -190,8 +191,9 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
 // warp); stores: 8 bytes of codes per channel and block as each block is done
 // (the four blocks of a 64-token item fill one 32-byte sector), one 4-byte
 // scale word per channel per item.
-// SR word for element (t, c): Philox counter (t*C + c) >> 2, so one call
-// serves the four channels of a row.
+// SR: one generator call per channel and 16-token block, keyed
+// idx0/16 + (token block) * C + channel; its four words serve the block's
+// sixteen tokens, four per stochastic-rounding conversion.
 // ---------------------------------------------------------------------------
 template <bool RHT, bool SR, bool NARROW>
 __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
@@ -214,7 +216,6 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
   const int64_t ng = C >> 2;
   const int64_t items = nq * ng;
   const int64_t half_r = R >> 1;
-  const uint64_t cq = static_cast<uint64_t>(C) >> 2;
   // item it = (token quad it / ng, channel group it % ng), kept incrementally
   const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x, step_q = step / ng, step_r = step - step_q * ng;
@@ -230,9 +231,6 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
     uint32_t sfw[4] = {0u, 0u, 0u, 0u};
     for (int tb = 0; tb < nb; ++tb) {
       const int64_t tbase = t0 + 16 * tb;
-      // SR counter of (tbase, c0): its element index in the whole tensor / 4
-      // (C, c0 and idx0 are multiples of 4, so row i adds i * C/4 exactly)
-      const uint64_t gq = static_cast<uint64_t>(tbase * C + c0 + idx0) >> 2;
       // v[p][i]: channels c0 + 2p (first) and c0 + 2p + 1 (second) at token tbase + i,
       // as FP32 pairs, so the transform and the scaling run as packed instructions
       float2 v[2][16];
@@ -271,28 +269,32 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
         r[c] = bs.r;
         sfw[c] |= bs.sf << (8 * tb);
       }
+      // y = v * r with the true sign (the register's, flipped where neg[i])
       const float2 r0 = make_float2(r[0], r[1]), r1 = make_float2(r[2], r[3]);
+      const float2 rn0 = make_float2(-r[0], -r[1]), rn1 = make_float2(-r[2], -r[3]);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        if (SR) {
-          // y = v * r, then the SR decision on |y| with the true sign (register sign, flipped by neg[i])
-          const float2 y0 = __fmul2_rn(v[0][i], r0), y1 = __fmul2_rn(v[1][i], r1);
-          const u32x4 w = sr_words<NARROW>(gq + i * cq, kDomainColSR, k0, k1);
-          if (neg[i]) {
-            v[0][i] = sr_magnitude2<true>(y0, w.x, w.y);
-            v[1][i] = sr_magnitude2<true>(y1, w.z, w.w);
-          } else {
-            v[0][i] = sr_magnitude2<false>(y0, w.x, w.y);
-            v[1][i] = sr_magnitude2<false>(y1, w.z, w.w);
-          }
-        } else {
-          const float2 rn0 = make_float2(-r[0], -r[1]), rn1 = make_float2(-r[2], -r[3]);
-          v[0][i] = __fmul2_rn(v[0][i], neg[i] ? rn0 : r0);
-          v[1][i] = __fmul2_rn(v[1][i], neg[i] ? rn1 : r1);
+        v[0][i] = __fmul2_rn(v[0][i], neg[i] ? rn0 : r0);
+        v[1][i] = __fmul2_rn(v[1][i], neg[i] ? rn1 : r1);
+      }
+      if (SR) {
+        // one generator call per channel and block: idx0/16 + (token block) * C + channel
+        const uint64_t gb = (static_cast<uint64_t>(idx0) >> 4) + static_cast<uint64_t>(tbase >> 4) * C +
+                            static_cast<uint64_t>(c0);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const u32x4 w = sr_words<NARROW>(gb + c, kDomainColSR, k0, k1);
+          const float2* u = v[c >> 1];
+          auto e = [&](int i) { return (c & 1) ? u[i].y : u[i].x; };
+          const uint32_t lo = sr_e2m1x4(e(0), e(1), e(2), e(3), w.x) | (sr_e2m1x4(e(4), e(5), e(6), e(7), w.y) << 16);
+          const uint32_t hi =
+              sr_e2m1x4(e(8), e(9), e(10), e(11), w.z) | (sr_e2m1x4(e(12), e(13), e(14), e(15), w.w) << 16);
+          reinterpret_cast<uint2*>(data + (c0 + c) * half_r + t0 / 2)[tb] =
+              make_uint2(clear_negative_zero(lo), clear_negative_zero(hi));
         }
       }
 #pragma unroll
-      for (int p = 0; p < 2; ++p) {
+      for (int p = 0; p < 2 && !SR; ++p) {
         const float2* w = v[p];
         const uint32_t a0 = clear_negative_zero(
             f32x8_to_e2m1x8(w[0].x, w[1].x, w[2].x, w[3].x, w[4].x, w[5].x, w[6].x, w[7].x));
@@ -758,6 +760,53 @@ cudaError_t selftest_div6(unsigned long long* bad_quotients, unsigned long long*
   return cudaSuccess;
 }
 
+// Self-test of the stochastic-rounding conversion against the rule it is
+// used for (sr_e2m1x4): for value i of a spread of magnitudes in [0, 6.5)
+// (every binade, arbitrary low bits, alternating signs), each of the four
+// lanes and every 16-bit draw x, the word is built so that the lane draws
+// exactly x, and the lane's code must be the upper neighbour iff
+// x + floor(p * 2^16) >= 2^16 (p the fractional position; floor(p * 2^16) is
+// exact in FP32).  Counts the codes that differ.
+constexpr int kSrTestValues = 8192;
+__device__ unsigned long long g_sr_test[2];
+
+__device__ __forceinline__ uint32_t rev16_bits(uint32_t x) { return __brev(x) >> 16; }
+
+__global__ void sr_selftest_kernel() {
+  const int vi = blockIdx.x >> 2, q = blockIdx.x & 3;
+  const uint32_t bits = static_cast<uint32_t>((0x40D00000ull * vi) / kSrTestValues) | ((vi & 1) ? 0x80000000u : 0u);
+  const float y = __uint_as_float(bits), a = fabsf(y);
+  const float step = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
+  const float lo = a >= 6.0f ? 6.0f : floorf(a / step) * step;
+  const float hi = a >= 6.0f ? 6.0f : fminf(lo + step, 6.0f);
+  const float fl = a >= 6.0f ? 0.0f : floorf(__fmul_rn(__fdiv_rn(a - lo, step), 65536.0f));   // floor(p * 2^16)
+  const float grid[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  unsigned long long bad = 0;
+  for (uint32_t x = threadIdx.x; x < 65536u; x += blockDim.x) {
+    const uint32_t d = (q & 1) ? rev16_bits(x) : x;   // the 16 bits the lane reads, in word order
+    const uint32_t word = (q < 2) ? ((d >> 8) << 16) | (d & 0xFFu) : ((d >> 8) << 24) | ((d & 0xFFu) << 8);
+    const uint32_t codes = sr_e2m1x4(y, y, y, y, word);
+    const float got = grid[(codes >> (4 * q)) & 7u];
+    const float want = (static_cast<float>(x) + fl >= 65536.0f) ? hi : lo;
+    if (got != want) ++bad;
+  }
+  if (bad) atomicAdd(&g_sr_test[0], bad);
+  if (threadIdx.x == 0) atomicAdd(&g_sr_test[1], 65536ull);
+}
+
+cudaError_t selftest_sr(unsigned long long* mismatches, unsigned long long* checked) {
+  const unsigned long long zero[2] = {0ull, 0ull};
+  cudaError_t e = cudaMemcpyToSymbol(g_sr_test, zero, sizeof(zero));
+  if (e != cudaSuccess) return e;
+  sr_selftest_kernel<<<kSrTestValues * 4, 256>>>();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  unsigned long long out[2];
+  if ((e = cudaMemcpyFromSymbol(out, g_sr_test, sizeof(out))) != cudaSuccess) return e;
+  *mismatches = out[0];
+  *checked = out[1];
+  return cudaSuccess;
+}
+
 cudaError_t launch_sf_pad_zero(void* scales, int64_t R, int64_t S, cudaStream_t s) {
   const int64_t Rp = (R + 127) / 128 * 128, Sp = (S + 3) / 4 * 4;
   if (Rp == R && Sp == S) return cudaSuccess;
@@ -787,7 +836,7 @@ cudaError_t launch_quant_row(const void* x, int64_t R, int64_t C, int64_t ld, co
   auto* d = static_cast<uint8_t*>(data);
   auto* f = static_cast<uint8_t*>(scales);
   if (sr)
-    if (idx0 + R * C < (int64_t(1) << 34))  // element index / 4 fits in 32 bits
+    if (idx0 + R * C < (int64_t(1) << 36))  // every block counter (element index / 16) fits in 32 bits
       quant_row_kernel<true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
     else
       quant_row_kernel<true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
@@ -808,7 +857,7 @@ cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, co
   auto* xs = static_cast<const uint16_t*>(x);
   auto* d = static_cast<uint8_t*>(data);
   auto* f = static_cast<uint8_t*>(scales);
-  const bool narrow = idx0 + R * C < (int64_t(1) << 34);  // element index / 4 fits in 32 bits
+  const bool narrow = idx0 + R * C < (int64_t(1) << 36);  // every block counter fits in 32 bits
   if (rht && sr && narrow)
     quant_col_kernel<true, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else if (rht && sr)

@@ -144,17 +144,18 @@ def test_data_parallel_linear_two_ranks_equal_one_process(tmp_path):
         assert np.all(np.abs(got - ref) <= tol), f"dW rank {rank}: {np.sum(np.abs(got - ref) > tol)} outside"
 
 
-@pytest.mark.parametrize("row0", [(1 << 34) // 320 - 16, (1 << 34) // 320 + 16, 1 << 30])
-def test_row_block_past_index_2_34(row0):
-    # element indices / 4 of these blocks pass 2^32 (the first straddles it), so
-    # the launchers pick the general SR kernels, whose Philox counter keeps a
-    # high word; codes and scales must equal the oracle's for the same offset
+@pytest.mark.parametrize("row0", [(1 << 36) // 320 - 16, (1 << 36) // 320 + 16, 1 << 32])
+def test_row_block_past_index_2_36(row0):
+    # the block counters (element index / 16) of these rows pass 2^32 (the
+    # first row block straddles it), so the launchers pick the general SR
+    # kernels, whose Philox counter keeps a high word; codes and scales must
+    # equal the oracle's for the same offset
     row0 -= row0 % 16
     x = synth.gradients(64, 320, 43)
     a, ar = O.amax(x), O.amax_rht(x)
     xd = dev(x)
     a_dev, ar_dev = api.amax(xd), api.amax(xd, rht=True)
-    assert row0 * 320 + 64 * 320 >= 1 << 34
+    assert row0 * 320 + 64 * 320 >= 1 << 36
     qr, _ = api.quantize(xd, api.ROW, a_dev, sr=True, seed=11, row0=row0)
     assert_q_equal(qr, *O.quantize_row(x, a, sr=True, seed=11, row0=row0), a, f"row sr row0={row0}")
     _, qc = api.quantize(xd, api.COL, a_dev, sr=True, seed=11, row0=row0)
