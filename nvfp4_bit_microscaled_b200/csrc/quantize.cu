@@ -184,18 +184,20 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
 }
 
 // ---------------------------------------------------------------------------
-// Column-wise 1x16 along R (the tokens: K of the Wgrad GEMM), transposed
-// output.  Thread item: 64 tokens x 4 channels.  Each 16-token block of a
-// channel is optionally rotated by Q = 1/4 H16 diag(s) before it is scaled.
-// Loads: 16 rows x 8 bytes per block (coalesced along the row across the
-// warp); stores: 8 bytes of codes per channel and block as each block is done
-// (the four blocks of a 64-token item fill one 32-byte sector), one 4-byte
-// scale word per channel per item.
+// Column-wise 1x16 along R (the tokens: K of the Wgrad GEMM) with stochastic
+// rounding, transposed output.  Thread item: 64 tokens x 2 channels.  Each
+// 16-token block of a channel is optionally rotated by Q = 1/4 H16 diag(s)
+// before it is scaled.  Loads: 16 rows x 4 bytes per block (128 coalesced
+// bytes per row across the warp).  The item's codes stay in registers and go
+// out once per item: a channel's 64 tokens are one 32-byte sector, written
+// with two 16-byte stores, which halves the scattered store transactions of
+// writing each block's 8 bytes as it is done.  One 4-byte scale word per
+// channel per item.
 // SR: one generator call per channel and 16-token block, keyed
 // idx0/16 + (token block) * C + channel; its four words serve the block's
 // sixteen tokens, four per stochastic-rounding conversion.
 // ---------------------------------------------------------------------------
-template <bool RHT, bool SR, bool NARROW>
+template <bool RHT, bool NARROW>
 __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
                                                              int64_t ld, const float* __restrict__ amax_dev,
                                                              uint32_t k0, uint32_t k1, int64_t idx0,
@@ -213,10 +215,10 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
   __syncthreads();
   const int64_t S = R >> 4;
   const int64_t nq = (S + 3) >> 2;
-  const int64_t ng = C >> 2;
+  const int64_t ng = C >> 1;
   const int64_t items = nq * ng;
   const int64_t half_r = R >> 1;
-  // item it = (token quad it / ng, channel group it % ng), kept incrementally
+  // item it = (token quad it / ng, channel pair it % ng), kept incrementally
   const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x, step_q = step / ng, step_r = step - step_q * ng;
   int64_t q_next = first / ng, g_next = first - q_next * ng;
@@ -226,90 +228,73 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
     g_next += step_r;
     q_next += step_q;
     if (g_next >= ng) g_next -= ng, ++q_next;
-    const int64_t c0 = g * 4, t0 = q * 64;
+    const int64_t c0 = g * 2, t0 = q * 64;
     const int nb = static_cast<int>((S - 4 * q) < 4 ? (S - 4 * q) : 4);
-    uint32_t sfw[4] = {0u, 0u, 0u, 0u};
-    for (int tb = 0; tb < nb; ++tb) {
-      const int64_t tbase = t0 + 16 * tb;
-      // v[p][i]: channels c0 + 2p (first) and c0 + 2p + 1 (second) at token tbase + i,
-      // as FP32 pairs, so the transform and the scaling run as packed instructions
-      float2 v[2][16];
+    uint32_t sfw[2] = {0u, 0u};
+    uint2 codes[2][4];   // the item's codes, per channel and block, stored once per item
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint2 raw = __ldcs(reinterpret_cast<const uint2*>(x + (tbase + i) * ld + c0));
-        v[0][i] = bf16x2_to_f32x2(raw.x);
-        v[1][i] = bf16x2_to_f32x2(raw.y);
-      }
+    for (int tb = 0; tb < 4; ++tb) {
+      if (tb >= nb) break;
+      const int64_t tbase = t0 + 16 * tb;
+      // v[i]: channels c0 (first) and c0 + 1 (second) at token tbase + i, as an
+      // FP32 pair, so the transform and the scaling run as packed instructions
+      float2 v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        v[i] = bf16x2_to_f32x2(__ldcs(reinterpret_cast<const unsigned int*>(x + (tbase + i) * ld + c0)));
       bool neg[16];   // true value of element i = -register (the RHT's signs, tracked at compile time)
 #pragma unroll
       for (int i = 0; i < 16; ++i) neg[i] = false;
-      float m[4];
+      float m0, m1;
       if (RHT) {
-        bool neg1[16];
-        fwht16_x2(v[0], neg);
-        fwht16_x2(v[1], neg1);   // the same compile-time signs
+        fwht16_x2(v, neg);
         // the 1/4 commutes with the maximum (exact power of two, monotone)
-        m[0] = __fmul_rn(absmax16<false>(v[0]), 0.25f);
-        m[1] = __fmul_rn(absmax16<true>(v[0]), 0.25f);
-        m[2] = __fmul_rn(absmax16<false>(v[1]), 0.25f);
-        m[3] = __fmul_rn(absmax16<true>(v[1]), 0.25f);
+        m0 = __fmul_rn(absmax16<false>(v), 0.25f);
+        m1 = __fmul_rn(absmax16<true>(v), 0.25f);
         const float2 q4 = make_float2(0.25f, 0.25f);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[0][i] = __fmul2_rn(v[0][i], q4), v[1][i] = __fmul2_rn(v[1][i], q4);
+        for (int i = 0; i < 16; ++i) v[i] = __fmul2_rn(v[i], q4);
       } else {
-        m[0] = absmax16<false>(v[0]);
-        m[1] = absmax16<true>(v[0]);
-        m[2] = absmax16<false>(v[1]);
-        m[3] = absmax16<true>(v[1]);
+        m0 = absmax16<false>(v);
+        m1 = absmax16<true>(v);
       }
-      float r[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const BlockScale bs = block_scale_t(m[c], s_enc, r_tbl);
-        r[c] = bs.r;
-        sfw[c] |= bs.sf << (8 * tb);
-      }
+      const BlockScale b0 = block_scale_t(m0, s_enc, r_tbl), b1 = block_scale_t(m1, s_enc, r_tbl);
+      sfw[0] |= b0.sf << (8 * tb);
+      sfw[1] |= b1.sf << (8 * tb);
       // y = v * r with the true sign (the register's, flipped where neg[i])
-      const float2 r0 = make_float2(r[0], r[1]), r1 = make_float2(r[2], r[3]);
-      const float2 rn0 = make_float2(-r[0], -r[1]), rn1 = make_float2(-r[2], -r[3]);
+      const float2 rp = make_float2(b0.r, b1.r), rn = make_float2(-b0.r, -b1.r);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        v[0][i] = __fmul2_rn(v[0][i], neg[i] ? rn0 : r0);
-        v[1][i] = __fmul2_rn(v[1][i], neg[i] ? rn1 : r1);
-      }
-      if (SR) {
-        // one generator call per channel and block: idx0/16 + (token block) * C + channel
-        const uint64_t gb = (static_cast<uint64_t>(idx0) >> 4) + static_cast<uint64_t>(tbase >> 4) * C +
-                            static_cast<uint64_t>(c0);
+      for (int i = 0; i < 16; ++i) v[i] = __fmul2_rn(v[i], neg[i] ? rn : rp);
+      // one generator call per channel and block: idx0/16 + (token block) * C + channel
+      const uint64_t gb = (static_cast<uint64_t>(idx0) >> 4) + static_cast<uint64_t>(tbase >> 4) * C +
+                          static_cast<uint64_t>(c0);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const u32x4 w = sr_words<NARROW>(gb + c, kDomainColSR, k0, k1);
-          const float2* u = v[c >> 1];
-          auto e = [&](int i) { return (c & 1) ? u[i].y : u[i].x; };
-          const uint32_t lo = sr_e2m1x4(e(0), e(1), e(2), e(3), w.x) | (sr_e2m1x4(e(4), e(5), e(6), e(7), w.y) << 16);
-          const uint32_t hi =
-              sr_e2m1x4(e(8), e(9), e(10), e(11), w.z) | (sr_e2m1x4(e(12), e(13), e(14), e(15), w.w) << 16);
-          reinterpret_cast<uint2*>(data + (c0 + c) * half_r + t0 / 2)[tb] =
-              make_uint2(clear_negative_zero(lo), clear_negative_zero(hi));
-        }
-      }
-#pragma unroll
-      for (int p = 0; p < 2 && !SR; ++p) {
-        const float2* w = v[p];
-        const uint32_t a0 = clear_negative_zero(
-            f32x8_to_e2m1x8(w[0].x, w[1].x, w[2].x, w[3].x, w[4].x, w[5].x, w[6].x, w[7].x));
-        const uint32_t a1 = clear_negative_zero(
-            f32x8_to_e2m1x8(w[8].x, w[9].x, w[10].x, w[11].x, w[12].x, w[13].x, w[14].x, w[15].x));
-        const uint32_t b0 = clear_negative_zero(
-            f32x8_to_e2m1x8(w[0].y, w[1].y, w[2].y, w[3].y, w[4].y, w[5].y, w[6].y, w[7].y));
-        const uint32_t b1 = clear_negative_zero(
-            f32x8_to_e2m1x8(w[8].y, w[9].y, w[10].y, w[11].y, w[12].y, w[13].y, w[14].y, w[15].y));
-        reinterpret_cast<uint2*>(data + (c0 + 2 * p) * half_r + t0 / 2)[tb] = make_uint2(a0, a1);
-        reinterpret_cast<uint2*>(data + (c0 + 2 * p + 1) * half_r + t0 / 2)[tb] = make_uint2(b0, b1);
+      for (int c = 0; c < 2; ++c) {
+        const u32x4 w = sr_words<NARROW>(gb + c, kDomainColSR, k0, k1);
+        auto e = [&](int i) { return c ? v[i].y : v[i].x; };
+        const uint32_t lo = sr_e2m1x4(e(0), e(1), e(2), e(3), w.x) | (sr_e2m1x4(e(4), e(5), e(6), e(7), w.y) << 16);
+        const uint32_t hi =
+            sr_e2m1x4(e(8), e(9), e(10), e(11), w.z) | (sr_e2m1x4(e(12), e(13), e(14), e(15), w.w) << 16);
+        codes[c][tb] = make_uint2(clear_negative_zero(lo), clear_negative_zero(hi));
       }
     }
+    // a channel's 64 tokens are 32 contiguous code bytes: two 16-byte stores
+    // where they are 16-byte aligned (channel rows of R/2 bytes start on
+    // 16-byte boundaries when R % 32 == 0); otherwise, and for a last item of
+    // fewer than four blocks, block by block
 #pragma unroll
-    for (int c = 0; c < 4; ++c) *reinterpret_cast<uint32_t*>(sf + sf_offset(c0 + c, 4 * q, sp)) = sfw[c];
+    for (int c = 0; c < 2; ++c) {
+      uint8_t* dst = data + (c0 + c) * half_r + t0 / 2;
+      if (nb == 4 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0u) {
+        reinterpret_cast<uint4*>(dst)[0] = make_uint4(codes[c][0].x, codes[c][0].y, codes[c][1].x, codes[c][1].y);
+        reinterpret_cast<uint4*>(dst)[1] = make_uint4(codes[c][2].x, codes[c][2].y, codes[c][3].x, codes[c][3].y);
+      } else {
+#pragma unroll
+        for (int tb = 0; tb < 4; ++tb)
+          if (tb < nb) reinterpret_cast<uint2*>(dst)[tb] = codes[c][tb];
+      }
+      *reinterpret_cast<uint32_t*>(sf + sf_offset(c0 + c, 4 * q, sp)) = sfw[c];
+    }
   }
 }
 
@@ -851,7 +836,8 @@ cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, co
                              int sr, uint64_t seed, int64_t idx0, void* data, void* scales, float* gs_out,
                              int num_sms, cudaStream_t s) {
   const int64_t S = R / 16, sp = (S + 3) / 4 * 4;
-  const int64_t items = ((S + 3) / 4) * (C / 4);
+  // items: 64 tokens x 2 channels (SR), 64 tokens x 4 channels (round to nearest)
+  const int64_t items = ((S + 3) / 4) * (C / (sr ? 2 : 4));
   const int grid = grid_for(items, 256, num_sms, 8);
   const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
   auto* xs = static_cast<const uint16_t*>(x);
@@ -859,15 +845,15 @@ cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, co
   auto* f = static_cast<uint8_t*>(scales);
   const bool narrow = idx0 + R * C < (int64_t(1) << 36);  // every block counter fits in 32 bits
   if (rht && sr && narrow)
-    quant_col_kernel<true, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
+    quant_col_kernel<true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else if (rht && sr)
-    quant_col_kernel<true, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
+    quant_col_kernel<true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else if (rht)
     quant_col_rn_kernel<true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, d, f, sp, gs_out);
   else if (sr && narrow)
-    quant_col_kernel<false, true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
+    quant_col_kernel<false, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else if (sr)
-    quant_col_kernel<false, true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
+    quant_col_kernel<false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
   else
     quant_col_rn_kernel<false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, d, f, sp, gs_out);
   cudaError_t e = cudaGetLastError();
