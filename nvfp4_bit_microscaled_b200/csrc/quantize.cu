@@ -184,8 +184,8 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
 }
 
 // ---------------------------------------------------------------------------
-// Column-wise 1x16 along R (the tokens: K of the Wgrad GEMM) with stochastic
-// rounding, transposed output.  Thread item: 64 tokens x 2 channels.  Each
+// Column-wise 1x16 along R (the tokens: K of the Wgrad GEMM), round to nearest
+// or stochastic, transposed output.  Thread item: 64 tokens x 2 channels.  Each
 // 16-token block of a channel is optionally rotated by Q = 1/4 H16 diag(s)
 // before it is scaled.  Loads: 16 rows x 4 bytes per block (128 coalesced
 // bytes per row across the warp).  The item's codes stay in registers and go
@@ -193,11 +193,12 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
 // with two 16-byte stores, which halves the scattered store transactions of
 // writing each block's 8 bytes as it is done.  One 4-byte scale word per
 // channel per item.
-// SR: one generator call per channel and 16-token block, keyed
+// The RHT copy of X for wgrad (round to nearest) and the dY copy (SR) both
+// run here.  SR: one generator call per channel and 16-token block, keyed
 // idx0/16 + (token block) * C + channel; its four words serve the block's
 // sixteen tokens, four per stochastic-rounding conversion.
 // ---------------------------------------------------------------------------
-template <bool RHT, bool NARROW>
+template <bool RHT, bool SR, bool NARROW>
 __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
                                                              int64_t ld, const float* __restrict__ amax_dev,
                                                              uint32_t k0, uint32_t k1, int64_t idx0,
@@ -265,16 +266,21 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
       const float2 rp = make_float2(b0.r, b1.r), rn = make_float2(-b0.r, -b1.r);
 #pragma unroll
       for (int i = 0; i < 16; ++i) v[i] = __fmul2_rn(v[i], neg[i] ? rn : rp);
-      // one generator call per channel and block: idx0/16 + (token block) * C + channel
+      // SR: one generator call per channel and block, idx0/16 + (token block) * C + channel
       const uint64_t gb = (static_cast<uint64_t>(idx0) >> 4) + static_cast<uint64_t>(tbase >> 4) * C +
                           static_cast<uint64_t>(c0);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        const u32x4 w = sr_words<NARROW>(gb + c, kDomainColSR, k0, k1);
         auto e = [&](int i) { return c ? v[i].y : v[i].x; };
-        const uint32_t lo = sr_e2m1x4(e(0), e(1), e(2), e(3), w.x) | (sr_e2m1x4(e(4), e(5), e(6), e(7), w.y) << 16);
-        const uint32_t hi =
-            sr_e2m1x4(e(8), e(9), e(10), e(11), w.z) | (sr_e2m1x4(e(12), e(13), e(14), e(15), w.w) << 16);
+        uint32_t lo, hi;
+        if (SR) {
+          const u32x4 w = sr_words<NARROW>(gb + c, kDomainColSR, k0, k1);
+          lo = sr_e2m1x4(e(0), e(1), e(2), e(3), w.x) | (sr_e2m1x4(e(4), e(5), e(6), e(7), w.y) << 16);
+          hi = sr_e2m1x4(e(8), e(9), e(10), e(11), w.z) | (sr_e2m1x4(e(12), e(13), e(14), e(15), w.w) << 16);
+        } else {
+          lo = f32x8_to_e2m1x8(e(0), e(1), e(2), e(3), e(4), e(5), e(6), e(7));
+          hi = f32x8_to_e2m1x8(e(8), e(9), e(10), e(11), e(12), e(13), e(14), e(15));
+        }
         codes[c][tb] = make_uint2(clear_negative_zero(lo), clear_negative_zero(hi));
       }
     }
@@ -295,97 +301,6 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
       }
       *reinterpret_cast<uint32_t*>(sf + sf_offset(c0 + c, 4 * q, sp)) = sfw[c];
     }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Column-wise 1x16 with round-to-nearest (the RHT copy of X for wgrad, and the
-// plain column copy): the same item, layout and arithmetic as quant_col_kernel
-// without SR, restructured for memory-level parallelism.  These copies are
-// bound by load latency, not by any pipe: the kernel above issues a block's
-// sixteen row loads only after it finished the previous block.  Here the
-// sixteen 8-byte loads of block b + 1 are issued before block b is computed
-// (two register buffers), and a block's four channels are unpacked and
-// processed one at a time, which keeps that second buffer within the
-// register budget of two CTAs per SM.
-// ---------------------------------------------------------------------------
-template <bool RHT>
-__global__ void __launch_bounds__(256, 2) quant_col_rn_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
-                                                                int64_t ld, const float* __restrict__ amax_dev,
-                                                                uint8_t* __restrict__ data, uint8_t* __restrict__ sf,
-                                                                int64_t sp, float* __restrict__ gs_out) {
-  __shared__ float r_tbl[kRTableSize];
-  const float amax = __ldg(amax_dev);
-  const float s_enc = encode_scale(amax);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && gs_out) *gs_out = decode_scale(amax);
-  if (!isfinite(amax)) {
-    flag_copy(data, C, R >> 1, sf, R >> 4, sp);
-    return;
-  }
-  fill_r_table(r_tbl, s_enc);
-  __syncthreads();
-  const int64_t S = R >> 4;
-  const int64_t nq = (S + 3) >> 2;
-  const int64_t ng = C >> 2;
-  const int64_t items = nq * ng;
-  const int64_t half_r = R >> 1;
-  const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x, step_q = step / ng, step_r = step - step_q * ng;
-  int64_t q_next = first / ng, g_next = first - q_next * ng;
-
-  for (int64_t it = first; it < items; it += step) {
-    const int64_t q = q_next, g = g_next;
-    g_next += step_r;
-    q_next += step_q;
-    if (g_next >= ng) g_next -= ng, ++q_next;
-    const int64_t c0 = g * 4, t0 = q * 64;
-    const int nb = static_cast<int>((S - 4 * q) < 4 ? (S - 4 * q) : 4);
-    const uint16_t* src = x + t0 * ld + c0;
-    uint32_t sfw[4] = {0u, 0u, 0u, 0u};
-    // block tb of the item -> codes of its four channels, scale bytes into sfw
-    auto block = [&](const uint2 (&cur)[16], int tb) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {   // one channel at a time: 16 floats live
-        float v[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const uint32_t w = (c < 2) ? cur[i].x : cur[i].y;
-          v[i] = __uint_as_float((c & 1) ? (w & 0xFFFF0000u) : (w << 16));
-          if (RHT && rht_negates(i)) v[i] = -v[i];  // s_i x_i
-        }
-        float m = 0.0f;
-        if (RHT) {
-          m = __fmul_rn(fwht16_absmax<true>(v), 0.25f);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.25f);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
-        }
-        const BlockScale bs = block_scale_t(m, s_enc, r_tbl);
-        sfw[c] |= bs.sf << (8 * tb);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], bs.r);
-        reinterpret_cast<uint2*>(data + (c0 + c) * half_r + t0 / 2)[tb] = make_uint2(pack8(v), pack8(v + 8));
-      }
-    };
-    auto load = [&](uint2 (&dst)[16], int tb) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) dst[i] = __ldcs(reinterpret_cast<const uint2*>(src + (16 * tb + i) * ld));
-    };
-    uint2 bufa[16], bufb[16];
-    load(bufa, 0);
-#pragma unroll 1
-    for (int tb = 0; tb < nb; tb += 2) {   // blocks tb (bufa) and tb + 1 (bufb), each loaded one block ahead
-      if (tb + 1 < nb) load(bufb, tb + 1);
-      block(bufa, tb);
-      if (tb + 1 < nb) {
-        if (tb + 2 < nb) load(bufa, tb + 2);
-        block(bufb, tb + 1);
-      }
-    }
-#pragma unroll
-    for (int c = 0; c < 4; ++c) *reinterpret_cast<uint32_t*>(sf + sf_offset(c0 + c, 4 * q, sp)) = sfw[c];
   }
 }
 
@@ -836,26 +751,23 @@ cudaError_t launch_quant_col(const void* x, int64_t R, int64_t C, int64_t ld, co
                              int sr, uint64_t seed, int64_t idx0, void* data, void* scales, float* gs_out,
                              int num_sms, cudaStream_t s) {
   const int64_t S = R / 16, sp = (S + 3) / 4 * 4;
-  // items: 64 tokens x 2 channels (SR), 64 tokens x 4 channels (round to nearest)
-  const int64_t items = ((S + 3) / 4) * (C / (sr ? 2 : 4));
+  const int64_t items = ((S + 3) / 4) * (C / 2);   // 64 tokens x 2 channels
   const int grid = grid_for(items, 256, num_sms, 8);
   const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
   auto* xs = static_cast<const uint16_t*>(x);
   auto* d = static_cast<uint8_t*>(data);
   auto* f = static_cast<uint8_t*>(scales);
   const bool narrow = idx0 + R * C < (int64_t(1) << 36);  // every block counter fits in 32 bits
-  if (rht && sr && narrow)
-    quant_col_kernel<true, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
-  else if (rht && sr)
-    quant_col_kernel<true, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
-  else if (rht)
-    quant_col_rn_kernel<true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, d, f, sp, gs_out);
-  else if (sr && narrow)
-    quant_col_kernel<false, true><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
-  else if (sr)
-    quant_col_kernel<false, false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, gs_out);
-  else
-    quant_col_rn_kernel<false><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, d, f, sp, gs_out);
+#define NVFP4_COL(RHT_, SR_, NARROW_)                                                                   \
+  quant_col_kernel<RHT_, SR_, NARROW_><<<grid, 256, 0, s>>>(xs, R, C, ld, amax_dev, k0, k1, idx0, d, f, sp, \
+                                                            gs_out)
+  if (rht && sr && narrow) NVFP4_COL(true, true, true);
+  else if (rht && sr) NVFP4_COL(true, true, false);
+  else if (rht) NVFP4_COL(true, false, false);
+  else if (sr && narrow) NVFP4_COL(false, true, true);
+  else if (sr) NVFP4_COL(false, true, false);
+  else NVFP4_COL(false, false, false);
+#undef NVFP4_COL
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_sf_pad_zero(scales, C, S, s);
