@@ -272,6 +272,7 @@ class AloneTimer:
         out = fn()   # untimed: the call's first-use work (an output allocation, a descriptor) is done here
         times = []
         for _ in range(self.reps):
+            out = None   # the previous output goes back to the allocator's cache, so the call reuses it
             torch.cuda.synchronize()
             self.scratch.fill_(1)
             if self.hold_cycles:
