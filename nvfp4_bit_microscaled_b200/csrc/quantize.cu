@@ -312,7 +312,8 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const uint16_t* __res
 // channels of the 16 rows (8-byte loads, 256 coalesced bytes per row per warp)
 // and quantizes their column blocks from registers, two channels at a time as
 // FP32 pairs (RHT optional, signs tracked at compile time, as the SR column
-// kernel does; scaled by the column copy's amax); it also stages the band in
+// kernel does; scaled by the column copy's amax), storing a channel's codes of
+// two bands at a time (16 bytes); it also stages the band in
 // shared memory, from which lanes read the band's 16 x 8 row blocks of 16
 // channels (two 16-byte reads each) and quantize them as the row kernel does
 // (scaled by the row copy's amax).  A non-finite amax flags its copy (R25).
@@ -349,6 +350,22 @@ __global__ void __launch_bounds__(256, 2) quant_rowcol_kernel(
     const bool lane_ok = c0 < C;
     const int nb = static_cast<int>((S - 4 * q) < 4 ? (S - 4 * q) : 4);
     uint32_t sfw[4] = {0u, 0u, 0u, 0u};
+    // column codes of an even band wait for the next band: a channel's two
+    // bands go out as one 16-byte store (two 8-byte stores where unaligned)
+    uint2 prev[4] = {};
+    auto put = [&](int c, int tb, uint2 cur) {
+      if (tb & 1) {
+        uint8_t* dst = col_data + (c0 + c) * half_r + t0 / 2 + 16 * (tb >> 1);
+        if ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0u) {
+          *reinterpret_cast<uint4*>(dst) = make_uint4(prev[c].x, prev[c].y, cur.x, cur.y);
+        } else {
+          reinterpret_cast<uint2*>(dst)[0] = prev[c];
+          reinterpret_cast<uint2*>(dst)[1] = cur;
+        }
+      } else {
+        prev[c] = cur;
+      }
+    };
     for (int tb = 0; tb < nb; ++tb) {
       const int64_t tbase = t0 + 16 * tb;
       uint2 raw[16];
@@ -406,8 +423,8 @@ __global__ void __launch_bounds__(256, 2) quant_rowcol_kernel(
               f32x8_to_e2m1x8(v[0].y, v[1].y, v[2].y, v[3].y, v[4].y, v[5].y, v[6].y, v[7].y));
           const uint32_t e1 = clear_negative_zero(
               f32x8_to_e2m1x8(v[8].y, v[9].y, v[10].y, v[11].y, v[12].y, v[13].y, v[14].y, v[15].y));
-          reinterpret_cast<uint2*>(col_data + (c0 + 2 * p) * half_r + t0 / 2)[tb] = make_uint2(a0, a1);
-          reinterpret_cast<uint2*>(col_data + (c0 + 2 * p + 1) * half_r + t0 / 2)[tb] = make_uint2(e0, e1);
+          put(2 * p, tb, make_uint2(a0, a1));
+          put(2 * p + 1, tb, make_uint2(e0, e1));
         }
       }
       __syncwarp();
@@ -438,7 +455,10 @@ __global__ void __launch_bounds__(256, 2) quant_rowcol_kernel(
     }
     if (!flag_col && lane_ok) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) *reinterpret_cast<uint32_t*>(col_sf + sf_offset(c0 + c, 4 * q, col_sp)) = sfw[c];
+      for (int c = 0; c < 4; ++c) {
+        if (nb & 1) reinterpret_cast<uint2*>(col_data + (c0 + c) * half_r + t0 / 2)[nb - 1] = prev[c];
+        *reinterpret_cast<uint32_t*>(col_sf + sf_offset(c0 + c, 4 * q, col_sp)) = sfw[c];
+      }
     }
   }
 }
