@@ -109,12 +109,28 @@ class ClockSampler:
         self.source = None
         self.t0 = self.t1 = None
         self.proc = self.thread = None
+        self.nvml = None                  # (module, handle) once NVML answers
 
+    # A timed region of a few tens of milliseconds can pass before the sampling
+    # thread gets to run, so the region's two edges are also sampled from the
+    # calling thread (NVML only): the first just after the start mark, the
+    # last just before the end mark.
     def mark_start(self):
         self.t0 = time.time()
+        self._sample_now()
 
     def mark_end(self):
+        self._sample_now()
         self.t1 = time.time()
+
+    def _sample_now(self):
+        if self.nvml is None:
+            return
+        nv, h = self.nvml
+        try:
+            self._nvml_sample(nv, h)
+        except Exception:
+            pass
 
     # -- NVML
     def _nvml_handle(self):
@@ -128,18 +144,23 @@ class ClockSampler:
         idx = int(vis.split(",")[self.device]) if vis else self.device
         return pynvml, pynvml.nvmlDeviceGetHandleByIndex(idx)
 
-    def _nvml_loop(self, nv, h, stop):
+    def _nvml_sample(self, nv, h):
         reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
             nv.nvmlDeviceGetCurrentClocksThrottleReasons
         bits = [(n, getattr(nv, attr, v)) for n, attr, v in self.REASONS]
         clk_max = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-        while not stop.wait(self.period):
+        clk = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        r = reasons_fn(h)
+        self.samples.append((time.time(), float(clk), float(clk_max), {n for n, b in bits if r & b}))
+
+    def _nvml_loop(self, nv, h, stop):
+        while True:   # a sample first, then every period until stopped
             try:
-                clk = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                r = reasons_fn(h)
+                self._nvml_sample(nv, h)
             except Exception:
-                continue
-            self.samples.append((time.time(), float(clk), float(clk_max), {n for n, b in bits if r & b}))
+                pass
+            if stop.wait(self.period):
+                return
 
     # -- nvidia-smi
     def _smi_start(self):
@@ -177,6 +198,7 @@ class ClockSampler:
             return self
         try:
             nv, h = self._nvml_handle()
+            self.nvml = (nv, h)
             import threading
             self.stop = threading.Event()
             self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h, self.stop), daemon=True)

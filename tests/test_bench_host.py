@@ -100,6 +100,18 @@ def test_nvml_sampler_decodes_reason_bits():
     assert s["reasons"] == ["sw_power_cap"] and s["sm_mhz"] in (1480, 1500, 1520)
 
 
+def test_short_timed_region_still_gets_its_edge_samples():
+    # no sampling thread at all: the start and end marks sample NVML themselves
+    nv = _FakeNvml([1900, 1910], 0x4)
+    c = bench.ClockSampler(0)
+    c.source = "nvml"
+    c.nvml = (nv, None)
+    c.mark_start()
+    c.mark_end()
+    s = c.summary()
+    assert s["samples"] == 2 and s["sm_mhz"] == 1905.0 and s["reasons"] == ["sw_power_cap"]
+
+
 def test_gemm_profile_is_reported_only_for_the_profiled_source(tmp_path, monkeypatch):
     root = tmp_path
     (root / "profiles").mkdir()
