@@ -444,6 +444,33 @@ def test_row_offset_reaches_the_counter_high_word():
     assert crossed
 
 
+def test_column_blocks_key_their_own_counters_past_2_32():
+    # R11 for the column copy: the block of channel c and tokens 16tb.. of rows
+    # row0.. of a larger tensor keys g = row0*C/16 + tb*C + c; here g passes
+    # 2^32, and every code equals the rule applied to that block's draws
+    C, rows = 64, 32
+    row0 = (1 << 36) // C - 16           # a multiple of 16: blocks straddle counter 2^32
+    x = synth.gradients(rows, C, 34)
+    a = O.amax(x)
+    codes_t, sf_t = O.quantize_col(x, a, sr=True, seed=9, row0=row0)
+    S_enc = float(O.global_scales(a)[0])
+    xf = x.float().numpy()
+    crossed = below = False
+    for c in (0, 1, 31, 63):
+        for tb in range(rows // 16):
+            g = (row0 * C) // 16 + tb * C + c
+            crossed |= g >= 1 << 32
+            below |= g < 1 << 32
+            draws = O.sr_block_draws(9, g, 1)
+            sb = O.e4m3_decode(sf_t[c, tb])
+            for i in range(16):
+                v = np.float32(xf[tb * 16 + i, c])
+                y = v * (np.float32(S_enc) / np.float32(sb)) if sb else np.float32(0)
+                want = O.e2m1_encode_sr(float(y), int(draws[i])) if sb else 0
+                assert codes_t[c, tb * 16 + i] == want, (c, tb, i)
+    assert crossed and below
+
+
 # ----------------------------------------------------------------- non-finite inputs (R25)
 def test_amax_propagates_nan_and_inf_like_numpy():
     x = synth.normal(48, 64, 33, std=2.0)
