@@ -193,8 +193,10 @@ __global__ void __launch_bounds__(256, 4) quant_row_kernel(const uint16_t* __res
 // with two 16-byte stores, which halves the scattered store transactions of
 // writing each block's 8 bytes as it is done.  One 4-byte scale word per
 // channel per item.
-// The RHT copy of X for wgrad (round to nearest) and the dY copy (SR) both
-// run here.  SR: one generator call per channel and 16-token block, keyed
+// Every NVFP4_COL copy runs here: round to nearest (with or without the RHT)
+// and stochastic (the linear layer's RHT copy of dY; X's column copy comes
+// from the ROWCOL kernel).  SR: one generator call per channel and 16-token
+// block, keyed
 // idx0/16 + (token block) * C + channel; its four words serve the block's
 // sixteen tokens, four per stochastic-rounding conversion.
 // ---------------------------------------------------------------------------
